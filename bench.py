@@ -1,0 +1,407 @@
+#!/usr/bin/env python3
+"""Benchmark of the FP8-AMAX linear layer on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fp8amax|reference]
+                    [--workload c3|c2|c1] [--no-e2e] [--no-cpu-baseline]
+
+A step is one pass of the whole hot path over the Llama-2-70B-shaped workload
+(d 8192, ffn 28672, GQA QKV 8192->10240, 8192 tokens): for each of the four
+projections, amax + bias + E4M3/E5M2 cast of X, W and dY, then the fwd, dgrad
+and wgrad FP8 GEMMs.  Inputs are seeded synthetic tensors, resident in HBM when
+the timed region starts; every step touches several GB, far more than the
+126 MB L2, so no step finds the previous one's data in cache.
+
+`value` is the layer's fwd+bwd GEMM FLOPs per second of whole step (amax and
+casts included).  `e2e` is the same metric through the C ABI starting from
+pinned HOST buffers: each step copies X, W, dY in and Y, dX, dW back.  The
+`roofline` object is the dominant kernel (the FP8 GEMM) against the dense FP8
+tensor-core peak; `roofline_quant` the amax+cast kernels against HBM.
+`cpu_baseline` is the CPU oracle timed on a bounded sample of the same step.
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own replica of
+the step (the layer does not shard across GPUs here): weak scaling, `value` =
+all ranks' FLOPs / the slowest rank's time.  `--impl reference` times the CPU
+oracle instead (rank 0 only).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "FP8-AMAX linear fwd+bwd TFLOP/s (% FP8 peak); amax+cast GB/s (% HBM)"
+UNIT = "TFLOP/s"
+NOMINAL_FP8_OVER_BF16 = 2.0      # dense FP8 / dense BF16 tensor-core rate (4.5 / 2.25 PFLOP/s)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fp8amax", choices=["fp8amax", "reference"])
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="approximate CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value, device):
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) of SM clock and throttle reasons."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200", "--id=" + uuid],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "power_w_max": max(power), "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ the step
+class Workload:
+    def __init__(self, cid, device, seed_step=0):
+        import fp8_tensor_scaled_b200 as fp8
+        self.fp8 = fp8
+        self.cfg = workloads.CONFIGS[cid]
+        self.device = device
+        self.inputs, self.layers = [], []
+        for li, lin in enumerate(self.cfg.linears):
+            x, w, dy = workloads.linear_inputs(cid, li, step=seed_step, device=device)
+            self.inputs.append((x, w, dy))
+            m = self.cfg.margins[0]
+            self.layers.append(fp8.Fp8AmaxLinear(self.cfg.tokens, lin.in_features,
+                                                 lin.out_features, device, self.cfg.out_dtype,
+                                                 m, m, m))
+        self.flops = sum(l.flops() for l in self.layers)
+        # algorithmic bytes of amax + cast: read the input twice, write one FP8 byte
+        self.quant_bytes = sum((2 * t.element_size() + 1) * t.numel()
+                               for inp in self.inputs for t in inp)
+        self.kernels_per_step = len(self.layers) * (3 * 2 + 3)   # 3 x (amax + cast) + 3 GEMMs
+
+    def step(self, ev=None):
+        for i, (layer, (x, w, dy)) in enumerate(zip(self.layers, self.inputs)):
+            if ev is not None:
+                ev[i][0].record()
+            layer.quantize(x, w, dy)
+            if ev is not None:
+                ev[i][1].record()
+            layer.gemms()
+            if ev is not None:
+                ev[i][2].record()
+
+
+def run_fp8(args, world, rank, local):
+    device = torch.device("cuda", local)
+    cid = int(args.workload[1:])
+    wl = Workload(cid, device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(max(3, args.warmup)):
+        wl.step()
+    torch.cuda.synchronize(device)
+
+    nlin = len(wl.layers)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nlin)]
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    start.record(stream)
+    for s in range(args.steps):
+        wl.step(evs[s])
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    clocks = sampler.stop()
+    barrier(world)
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(world, ms_local, device)
+    quant_ms = sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps)
+                   for i in range(nlin))
+    gemm_ms = sum(evs[s][i][1].elapsed_time(evs[s][i][2]) for s in range(args.steps)
+                  for i in range(nlin))
+    per_linear_gemm_ms = [sum(evs[s][i][1].elapsed_time(evs[s][i][2])
+                              for s in range(args.steps)) / args.steps for i in range(nlin)]
+    res = dict(ms=ms, ms_local=ms_local, quant_ms=quant_ms, gemm_ms=gemm_ms,
+               per_linear_gemm_ms=per_linear_gemm_ms, clocks=clocks, wl=wl)
+
+    if not args.no_e2e:
+        res["e2e"] = run_e2e(args, wl, device, world)
+    return res
+
+
+def run_e2e(args, wl, device, world):
+    """Same step through the C ABI from pinned host buffers, copies timed."""
+    host_in = [tuple(t.cpu().pin_memory() for t in inp) for inp in wl.inputs]
+    host_out = [tuple(torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+                      for o in (l.y, l.dx, l.dw)) for l in wl.layers]
+    h2d = sum(t.numel() * t.element_size() for inp in host_in for t in inp)
+    d2h = sum(t.numel() * t.element_size() for out in host_out for t in out)
+    stream = torch.cuda.current_stream(device)
+
+    def one():
+        for (hx, hw, hdy), (x, w, dy) in zip(host_in, wl.inputs):
+            x.copy_(hx, non_blocking=True)
+            w.copy_(hw, non_blocking=True)
+            dy.copy_(hdy, non_blocking=True)
+        wl.step()
+        for layer, (hy, hdx, hdw) in zip(wl.layers, host_out):
+            hy.copy_(layer.y, non_blocking=True)
+            hdx.copy_(layer.dx, non_blocking=True)
+            hdw.copy_(layer.dw, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(device)
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        one()
+    b.record(stream)
+    b.synchronize()
+    ms = max_over_ranks(world, a.elapsed_time(b), device) / args.e2e_steps
+    return {"ms_per_step": ms, "h2d": h2d, "d2h": d2h}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(cid, seconds, device_inputs=None):
+    """Time the CPU oracle on a bounded sample of one step and extrapolate.
+
+    Sample: for every linear and pass, `r` full output rows of the fp64 oracle
+    matmul, plus amax + bias + cast of the first 2^22 elements of each input
+    tensor.  The whole-step CPU time is extrapolated linearly (the oracle's
+    cost is proportional to output rows and to elements)."""
+    import oracle
+    cfg = workloads.CONFIGS[cid]
+    g = torch.Generator().manual_seed(1)
+    n_q = 1 << 22
+    t_quant, n_quant_done, n_quant_total = 0.0, 0, 0
+    t_gemm, f_gemm_done = 0.0, 0
+    rows = 1
+    for li, lin in enumerate(cfg.linears):
+        T, In, Out = cfg.tokens, lin.in_features, lin.out_features
+        # small seeded stand-ins with the real K extents (the oracle's cost does
+        # not depend on the values)
+        for shape in ((T, In), (Out, In), (T, Out)):
+            n_quant_total += shape[0] * shape[1]
+            x = torch.randn(min(n_q, shape[0] * shape[1]), generator=g).to(torch.bfloat16)
+            t0 = time.perf_counter()
+            oracle.quantize(x, 0, 0)
+            t_quant += time.perf_counter() - t0
+            n_quant_done += x.numel()
+        xq = torch.randint(0, 120, (rows, In), generator=g, dtype=torch.uint8).numpy()
+        wq = torch.randint(0, 120, (Out, In), generator=g, dtype=torch.uint8).numpy()
+        dq = torch.randint(0, 120, (T, Out), generator=g, dtype=torch.uint8).numpy()
+        xfull = torch.randint(0, 120, (T, In), generator=g, dtype=torch.uint8).numpy()
+        # fwd rows: Y[r, :] needs X[r, :] and all of W
+        t0 = time.perf_counter()
+        oracle.linear(oracle.FWD, xq, 0, 0, wq, 0, 0, rows, In, Out, with_abs=False)
+        # dgrad rows: dX[r, :] needs dY[r, :] and all of W
+        oracle.linear(oracle.DGRAD, dq[:rows], 1, 0, wq, 0, 0, rows, In, Out, with_abs=False)
+        # wgrad rows: dW[o, :] for o < rows needs dY[:, o] and all of X
+        oracle.linear(oracle.WGRAD, dq[:, :16].copy(), 1, 0, xfull, 0, 0, T, In, 16,
+                      with_abs=False)
+        t_gemm += time.perf_counter() - t0
+        f_gemm_done += 2 * rows * In * Out + 2 * rows * Out * In + 2 * 16 * T * In
+    flops = cfg.flops_per_step()
+    est_gemm = t_gemm * flops / f_gemm_done
+    est_quant = t_quant * n_quant_total / n_quant_done
+    est_step = est_gemm + est_quant
+    sample = ("oracle on 1 output row of fwd and dgrad and 16 rows of wgrad per projection "
+              "(full K), plus amax+bias+cast of 2^22 elements of each of the 12 input tensors; "
+              "whole-step time extrapolated by FLOPs and by elements")
+    return {"value": flops / est_step / 1e12, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": sample, "sample_seconds": round(t_gemm + t_quant, 3),
+            "est_step_seconds": round(est_step, 1)}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle, timed as it stands (rank 0 only)."""
+    if rank != 0:
+        return 0
+    cid = int(args.workload[1:])
+    for _ in range(args.warmup):
+        oracle_sample(cid, args.cpu_seconds)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        r = oracle_sample(cid, args.cpu_seconds)
+        vals.append(r["value"])
+        secs.append(r["sample_seconds"])
+    v = statistics.median(vals)
+    cfg = workloads.CONFIGS[cid]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * cfg.flops_per_step() / (v * 1e12), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(cfg, args.gpus),
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                         "sample": r["sample"]},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(cfg, n):
+    return {"workload": cfg.name, "tokens": cfg.tokens,
+            "linears": ["%s %d->%d" % (l.name, l.in_features, l.out_features) for l in cfg.linears],
+            "passes": list(cfg.passes), "formats": "E4M3 X,W / E5M2 dY", "margin": cfg.margins[0],
+            "out_dtype": str(cfg.out_dtype).replace("torch.", ""),
+            "l2": "inputs larger than L2 (a step reads and writes several GB)",
+            "parallelism": "replicas x%d" % n}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        rc = run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "no CUDA device"}))
+        return 1
+    peaks, peak_src = load_peaks()
+    r = run_fp8(args, world, rank, local)
+    wl = r["wl"]
+    steps = args.steps
+    ms_step = r["ms"] / steps
+    total_flops = wl.flops * world
+    value = total_flops / (ms_step * 1e-3) / 1e12
+    gemm_tflops = wl.flops * steps / (r["gemm_ms"] * 1e-3) / 1e12
+    quant_gbs = wl.quant_bytes * steps / (r["quant_ms"] * 1e-3) / 1e9
+    fp8_peak = peaks["bf16_tflops_sustained"] * NOMINAL_FP8_OVER_BF16
+    hbm_peak = peaks["hbm_gbs"]
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8",
+        "data": "synthetic", "config": config_dict(wl.cfg, world),
+        "gemm_tflops": round(gemm_tflops, 2), "quant_gbs": round(quant_gbs, 1),
+        "per_linear_gemm_ms": [round(x, 4) for x in r["per_linear_gemm_ms"]],
+        "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 2), "peak": round(fp8_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp8_peak, 4), "traffic": None,
+                     "kernel": "fp8_gemm_kernel (fwd/dgrad/wgrad)",
+                     "peak_source": "%s bf16 sustained x %.0f (dense FP8/BF16 ratio)"
+                                    % (peak_src, NOMINAL_FP8_OVER_BF16)},
+        "roofline_quant": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm_peak,
+                           "unit": "GB/s", "frac": round(quant_gbs / hbm_peak, 4),
+                           "kernel": "amax_kernel + cast_kernel",
+                           "bytes_per_element": "2*s_in + 1", "peak_source": peak_src},
+        "clocks": r["clocks"],
+        "gpu_launches": wl.kernels_per_step * steps,
+    }
+    if "e2e" in r:
+        e = r["e2e"]
+        line["e2e"] = {"value": round(total_flops / (e["ms_per_step"] * 1e-3) / 1e12, 2),
+                       "unit": UNIT, "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                       "ms_per_step": round(e["ms_per_step"], 3)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample(int(args.workload[1:]), args.cpu_seconds)
+        line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,491 @@
+// gemm_sm100.cu — the FP8 matmuls of the FP8-AMAX linear layer on sm_100a.
+//
+// D[M,N] = (A[M,K] . B[N,K]^T) * 2^-(bias_a + bias_b), FP8 operands (E4M3 or
+// E5M2, any mix), fp32 accumulation in tensor memory, one RNE conversion to
+// BF16 or FP32 in the epilogue.  The three passes of a linear layer map to it
+// without any transpose copy (review page "Training and inference of large
+// language models using 8-bit floating point", "Proposed method": the matmul
+// runs on the scaled FP8 operands and its output is unscaled afterwards):
+//   fwd    Y  = X . W^T      A = X  [T,in]  K-major,  B = W [out,in] K-major
+//   dgrad  dX = dY . W       A = dY [T,out] K-major,  B = W [out,in] MN-major
+//   wgrad  dW = dY^T . X     A = dY [T,out] MN-major, B = X [T,in]   MN-major
+//
+// Design (one CTA per SM, persistent, warp-specialised):
+//   warp 0      TMA producer: 128x128 (A) and 256x128 (B) FP8 boxes, 128-byte
+//               swizzle, into a 4-stage shared-memory ring (48 KB per stage),
+//               completion tracked by mbarrier transaction counts.
+//   warp 1      TMEM allocator (512 columns = two 128x256 fp32 accumulators)
+//               and MMA issuer: one thread issues tcgen05.mma kind::f8f6f4,
+//               M=128 N=256 K=32, four per stage, and tcgen05.commit frees the
+//               stage / publishes a finished accumulator.
+//   warps 2-5   epilogue: tcgen05.ld 32x32b of the accumulator, multiply by the
+//               power of two 2^-(bias_a+bias_b), convert, store to global;
+//               double-buffered accumulators let it overlap the next tile's
+//               mainloop.
+// Tiles are visited in groups of `group_n` N-blocks (N fastest inside a group)
+// so that the CTAs running at the same time share A and B panels in L2.
+//
+// Every mbarrier wait is bounded in time.  A wait that runs out records its
+// site in a device error word, raises a block-wide abort flag, and every role
+// leaves its loop; the MMA thread and the producer then drain their own
+// in-flight tensor-core work and copies (again with bounded waits) before the
+// tensor memory is released and the block exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fp8amax {
+
+// Device error word: 0 or the site of the first bounded wait that ran out.
+static __device__ int g_device_error = 0;
+
+namespace {
+
+enum WaitSite : int {
+  kSiteProducerEmpty = 1,
+  kSiteMmaFull = 2,
+  kSiteMmaTmemEmpty = 3,
+  kSiteEpilogueTmemFull = 4,
+  kSiteDrain = 5,
+  kSiteSelfTest = 6,
+};
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s; a correct kernel waits microseconds
+constexpr uint64_t kDrainLimitNs = 100000000ull;   // 100 ms for draining after an abort
+
+__device__ __forceinline__ void record_device_error(int site) {
+  atomicCAS(&g_device_error, 0, site);
+}
+
+// Wait until the phase with the given parity has completed, for at most
+// `limit_ns`.  Returns false when the wait gave up: either the limit ran out
+// (the site is recorded and *abort raised) or another role raised *abort.
+// Called by ONE thread.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  volatile int* abort_flag, int site,
+                                                  uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      record_device_error(site);
+      return false;
+    }
+  }
+}
+
+constexpr int BM = 128;                 // UMMA M (one CTA)
+constexpr int BN = 256;                 // UMMA N
+constexpr int BK = 128;                 // K per stage: one 128-byte swizzle row of FP8
+constexpr int UK = 32;                  // K per tcgen05.mma of kind::f8f6f4
+constexpr int STAGES = 4;
+constexpr uint32_t A_BYTES = BM * BK;   // 16 KB
+constexpr uint32_t B_BYTES = BN * BK;   // 32 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 512;     // 2 accumulators x 256 fp32 columns
+constexpr int kThreads = 192;           // 6 warps
+constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1;
+constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + kNumBars * 8 + 16;
+
+struct Params {
+  int M, N, K;
+  int num_m_blocks, num_n_blocks, num_k_blocks, num_tiles;
+  int group_n;
+  uint32_t idesc;
+  const int32_t* bias_a;
+  const int32_t* bias_b;
+  void* d;
+  uint64_t wait_limit_ns;
+};
+
+// Shared-memory matrix descriptor (tcgen05 format): start address, leading
+// and stride byte offsets (all >> 4), descriptor version 1 at bit 46,
+// 128-byte swizzle (layout type 2) in bits 61-63.
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 2ull << 61;
+  return d;
+}
+
+// K-major operand (rows of 128 K-bytes, 8-row swizzle atoms of 1 KB):
+// SBO = 1024 between 8-row groups, LBO unused (16); sub-step k advances the
+// start address by 32 bytes inside the swizzle row.
+// MN-major operand (rows of 128 MN-bytes, one per K index): SBO = 1024 between
+// groups of 8 K rows, LBO = 16 KB between 128-wide MN chunks; sub-step k
+// advances by 32 K rows = 4 KB.
+template <bool kMN>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t stage_base, int k) {
+  if (kMN) return make_sdesc(stage_base + k * (UK * 128), BK * 128, 1024);
+  return make_sdesc(stage_base + k * UK, 16, 1024);
+}
+
+__device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
+  const int group_size = p.group_n * p.num_m_blocks;
+  const int g = t / group_size;
+  const int first_n = g * p.group_n;
+  const int gn = min(p.group_n, p.num_n_blocks - first_n);
+  const int r = t - g * group_size;
+  mb = r / gn;
+  nb = first_n + r % gn;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <bool kAMN, bool kBMN, bool kOutF32>
+__global__ void __launch_bounds__(kThreads, 1)
+fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                const __grid_constant__ CUtensorMap tmap_b, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);          // one arrival per epilogue warp
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ----------------------------- TMA producer -----------------------------
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed_mask = 0, armed_parity = 0;   // per stage: last armed phase
+    for (int t = blockIdx.x; t < p.num_tiles && !*abort_flag; t += gridDim.x) {
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      bool ok = true;
+      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, kSiteProducerEmpty,
+                               p.wait_limit_ns)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = full_bar(stage);
+        mbar_arrive_expect_tx(fb, STAGE_BYTES);
+        armed_mask |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
+        const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
+        const int k0 = kb * BK;
+        if (kAMN) tma_load_2d(a_dst, &tmap_a, fb, mb * BM, k0);
+        else      tma_load_2d(a_dst, &tmap_a, fb, k0, mb * BM);
+        if (kBMN) {
+          tma_load_2d(b_dst, &tmap_b, fb, nb * BN, k0);
+          tma_load_2d(b_dst + BK * 128, &tmap_b, fb, nb * BN + 128, k0);
+        } else {
+          tma_load_2d(b_dst, &tmap_b, fb, k0, nb * BN);
+        }
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+    // Every copy this thread issued completes its stage's full barrier; wait
+    // for the last one of each stage so that no copy is still landing in shared
+    // memory when the block exits (immediate in the normal case).
+    int never = 0;
+    for (int s = 0; s < STAGES; ++s)
+      if (armed_mask & (1u << s))
+        mbar_wait_bounded(full_bar(s), (armed_parity >> s) & 1u, &never, kSiteDrain, kDrainLimitNs);
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------ MMA issuer ------------------------------
+    int stage = 0;
+    uint32_t phase = 0;
+    int local = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      if (!mbar_wait_bounded(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, kSiteMmaTmemEmpty,
+                             p.wait_limit_ns))
+        break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      bool ok = true;
+      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+        if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, kSiteMmaFull, p.wait_limit_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + stage * A_BYTES);
+        const uint32_t b_base = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / UK; ++k) {
+          mma_f8f6f4(d_tmem, operand_desc<kAMN>(a_base, k), operand_desc<kBMN>(b_base, k), p.idesc,
+                     (kb | k) != 0 ? 1u : 0u);
+        }
+        mma_commit(empty_bar(stage));     // frees the stage once these MMAs have read it
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      mma_commit(tfull_bar(acc));         // accumulator complete
+    }
+    // Drain: the commit arrives only after every MMA this thread issued is done.
+    mma_commit(drain_bar);
+    int never = 0;
+    mbar_wait_bounded(drain_bar, 0, &never, kSiteDrain, kDrainLimitNs);
+  } else if (warp >= 2) {
+    // ------------------------------- epilogue -------------------------------
+    const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+    const int row_in_tile = quarter * 32 + lane;
+    const Pow2Scale sc = make_pow2_scale(-(*p.bias_a + *p.bias_b));
+    int local = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+      const int acc = local & 1;
+      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      int ok = 1;
+      if (lane == 0)
+        ok = mbar_wait_bounded(tfull_bar(acc), use & 1u, abort_flag, kSiteEpilogueTmemFull,
+                               p.wait_limit_ns) ? 1 : 0;
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      const int64_t row = static_cast<int64_t>(mb) * BM + row_in_tile;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int col0 = nb * BN + c * 32;
+        if (col0 >= p.N) break;                   // warp-uniform
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                               static_cast<uint32_t>(acc * BN + c * 32), r);
+        tmem_ld_wait();
+        if (row_ok) {
+          if (kOutF32) {
+            float* dst = static_cast<float*>(p.d) + row * p.N + col0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              if (col0 + 4 * j < p.N) {
+                float4 v;
+                v.x = apply_pow2(__uint_as_float(r[4 * j + 0]), sc);
+                v.y = apply_pow2(__uint_as_float(r[4 * j + 1]), sc);
+                v.z = apply_pow2(__uint_as_float(r[4 * j + 2]), sc);
+                v.w = apply_pow2(__uint_as_float(r[4 * j + 3]), sc);
+                *reinterpret_cast<float4*>(dst + 4 * j) = v;
+              }
+            }
+          } else {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.d) + row * p.N + col0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (col0 + 8 * j < p.N) {
+                uint4 v;
+                v.x = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 0]), sc),
+                                  apply_pow2(__uint_as_float(r[8 * j + 1]), sc));
+                v.y = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 2]), sc),
+                                  apply_pow2(__uint_as_float(r[8 * j + 3]), sc));
+                v.z = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 4]), sc),
+                                  apply_pow2(__uint_as_float(r[8 * j + 5]), sc));
+                v.w = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 6]), sc),
+                                  apply_pow2(__uint_as_float(r[8 * j + 7]), sc));
+                *reinterpret_cast<uint4*>(dst + 8 * j) = v;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// One thread waits on a barrier nothing completes; the bounded wait must give
+// up after `limit_ns`, record the self-test site and return.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbarrier_init();
+    mbar_wait_bounded(smem_u32(&bar), 0, &abort_flag, kSiteSelfTest, limit_ns);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Host side
+// ----------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D row-major uint8 tensor [outer, inner], box [box_outer, box_inner],
+// 128-byte swizzle, zero fill out of bounds.
+bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
+               uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int g_sm_count[64];
+
+int sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (g_sm_count[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    g_sm_count[dev] = n > 0 ? n : 148;
+  }
+  return g_sm_count[dev];
+}
+
+template <bool kAMN, bool kBMN, bool kOutF32>
+int launch_t(const GemmArgs& g, cudaStream_t s) {
+  CUtensorMap ta, tb;
+  const uint64_t M = g.M, N = g.N, K = g.K;
+  const bool ok_a = kAMN ? encode_2d(&ta, g.a, M, K, 128, BK) : encode_2d(&ta, g.a, K, M, BK, BM);
+  const bool ok_b = kBMN ? encode_2d(&tb, g.b, N, K, 128, BK) : encode_2d(&tb, g.b, K, N, BK, BN);
+  if (!ok_a || !ok_b) return FP8_ERR_CUDA;
+
+  Params p;
+  p.M = static_cast<int>(g.M);
+  p.N = static_cast<int>(g.N);
+  p.K = static_cast<int>(g.K);
+  p.num_m_blocks = (p.M + BM - 1) / BM;
+  p.num_n_blocks = (p.N + BN - 1) / BN;
+  p.num_k_blocks = (p.K + BK - 1) / BK;
+  p.num_tiles = p.num_m_blocks * p.num_n_blocks;
+  p.group_n = 8;
+  p.idesc = (1u << 4)                                      // D = fp32
+            | (static_cast<uint32_t>(g.a_fmt) << 7)       // A: 0 E4M3, 1 E5M2
+            | (static_cast<uint32_t>(g.b_fmt) << 10)      // B: 0 E4M3, 1 E5M2
+            | (static_cast<uint32_t>(kAMN) << 15)         // A major: 0 K, 1 MN
+            | (static_cast<uint32_t>(kBMN) << 16)         // B major
+            | (static_cast<uint32_t>(BN >> 3) << 17)      // N / 8
+            | (static_cast<uint32_t>(BM >> 4) << 24);     // M / 16
+  p.bias_a = g.bias_a;
+  p.bias_b = g.bias_b;
+  p.d = g.d;
+  p.wait_limit_ns = kWaitLimitNs;
+
+  static bool attr_set[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  auto kern = fp8_gemm_kernel<kAMN, kBMN, kOutF32>;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
+  kern<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, p);
+  return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_gemm(const GemmArgs& g, cudaStream_t s) {
+  // limits of the 32-bit tile arithmetic and of the TMA tensor map
+  if (g.M > (1LL << 31) - 1 - BM || g.N > (1LL << 31) - 1 - BN || g.K > (1LL << 31) - 1 - BK)
+    return FP8_ERR_UNSUPPORTED;
+  const int key = (g.a_mn_major ? 4 : 0) | (g.b_mn_major ? 2 : 0) | (g.d_fp32 ? 1 : 0);
+  switch (key) {
+    case 0: return launch_t<false, false, false>(g, s);
+    case 1: return launch_t<false, false, true>(g, s);
+    case 2: return launch_t<false, true, false>(g, s);
+    case 3: return launch_t<false, true, true>(g, s);
+    case 6: return launch_t<true, true, false>(g, s);
+    case 7: return launch_t<true, true, true>(g, s);
+    default: return FP8_ERR_UNSUPPORTED;   // MN-major A with K-major B: no pass uses it
+  }
+}
+
+cudaError_t launch_selftest_wait(uint64_t timeout_ns) {
+  selftest_wait_kernel<<<1, 32>>>(timeout_ns);
+  return cudaGetLastError();
+}
+
+int device_error_site(bool clear) {
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return -1;
+  if (clear && v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return -1;
+  }
+  return v;
+}
+
+}  // namespace fp8amax

@@ -1,0 +1,215 @@
+"""GPU parity of the FP8 linear passes (fwd, dgrad, wgrad) through the C ABI,
+against the oracle's fp64 matmul of the dequantised FP8 codes.
+
+Tolerance (per element): |gpu - ref| <= 1e-3 * sum|a*b| * 2^-(bA+bB) + 1 BF16 ulp
+(see tests/parity.py).  Small shapes are compared in full — ragged in every
+dimension against the 128 x 256 x 128 tiles — and the layer shapes of the
+GPT-111M, Llama-2-7B and Llama-2-70B workloads are compared on sampled
+elements and whole 128-row blocks, in the same launch configuration the
+benchmark times."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from parity import assert_gemm_close, codes_equal_nan_aware, to_f64, u8
+
+pytestmark = pytest.mark.gpu
+
+fp8 = pytest.importorskip("fp8_tensor_scaled_b200")
+DEV = "cuda"
+E4, E5 = fp8.E4M3, fp8.E5M2
+
+
+def _quant(x_cpu, fmt, margin):
+    """Device quantize + the oracle's own quantize of the same bytes."""
+    a, b, q = fp8.fp8_quantize(x_cpu.to(DEV), fmt, margin)
+    m_ref, b_ref, q_ref = oracle.quantize(x_cpu, fmt, margin)
+    assert int(b.item()) == b_ref
+    assert codes_equal_nan_aware(u8(q), q_ref.reshape(x_cpu.shape), fmt)
+    return q, b, q_ref.reshape(tuple(x_cpu.shape)), b_ref
+
+
+def _passes(x, w, dy, margins=(0, 0, 0), fx=E4, fw=E4, fdy=E5):
+    """Quantize and return everything the passes need (device and oracle sides)."""
+    qx, bx, rqx, rbx = _quant(x, fx, margins[0])
+    qw, bw, rqw, rbw = _quant(w, fw, margins[1])
+    out = dict(x=(qx, bx, rqx, rbx, fx), w=(qw, bw, rqw, rbw, fw))
+    if dy is not None:
+        out["dy"] = _quant(dy, fdy, margins[2]) + (fdy,)
+    return out
+
+
+def _run(pass_, Q, out_dtype):
+    qx, bx, _, _, fx = Q["x"]
+    qw, bw, _, _, fw = Q["w"]
+    if pass_ == oracle.FWD:
+        return fp8.fp8_linear_fwd(qx, fx, bx, qw, fw, bw, out_dtype=out_dtype)
+    qdy, bdy, _, _, fdy = Q["dy"]
+    if pass_ == oracle.DGRAD:
+        return fp8.fp8_linear_bwd_dgrad(qdy, fdy, bdy, qw, fw, bw, out_dtype=out_dtype)
+    return fp8.fp8_linear_bwd_wgrad(qdy, fdy, bdy, qx, fx, bx, out_dtype=out_dtype)
+
+
+def _oracle_args(pass_, Q):
+    _, _, rqx, rbx, fx = Q["x"]
+    _, _, rqw, rbw, fw = Q["w"]
+    if pass_ == oracle.FWD:
+        return rqx, fx, rbx, rqw, fw, rbw
+    _, _, rqdy, rbdy, fdy = Q["dy"]
+    if pass_ == oracle.DGRAD:
+        return rqdy, fdy, rbdy, rqw, fw, rbw
+    return rqdy, fdy, rbdy, rqx, fx, rbx
+
+
+def _compare_full(pass_, Q, T, In, Out, out_dtype, what):
+    y = _run(pass_, Q, out_dtype)
+    torch.cuda.synchronize()
+    ref, absref = oracle.linear(pass_, *_oracle_args(pass_, Q), T, In, Out)
+    return assert_gemm_close(to_f64(y), ref, absref, what)
+
+
+def _compare_sampled(pass_, Q, T, In, Out, out_dtype, what, n_samples=1 << 14, block_cols=2048):
+    y = _run(pass_, Q, out_dtype)
+    torch.cuda.synchronize()
+    R, C = y.shape
+    rng = np.random.default_rng(1000 + pass_ + R + C)
+    rows = rng.integers(0, R, n_samples)
+    cols = rng.integers(0, C, n_samples)
+    # corners and the last row / column (ragged tile edges)
+    rows = np.concatenate([rows, [0, R - 1, R - 1, 0]])
+    cols = np.concatenate([cols, [0, C - 1, 0, C - 1]])
+    # one whole 128-row block, first `block_cols` columns
+    rb = int(rng.integers(0, max(1, R // 128))) * 128
+    br, bc = np.meshgrid(np.arange(rb, min(rb + 128, R)), np.arange(min(block_cols, C)),
+                         indexing="ij")
+    rows = np.concatenate([rows, br.ravel()])
+    cols = np.concatenate([cols, bc.ravel()])
+    ref, absref = oracle.linear_entries(pass_, *_oracle_args(pass_, Q), T, In, Out, rows, cols)
+    got = to_f64(y)[rows, cols]
+    return assert_gemm_close(got, ref, absref, what)
+
+
+def _inputs(T, In, Out, seed, x_scale=1.0, w_scale=0.02, dy_scale=1e-4):
+    g = torch.Generator().manual_seed(seed)
+    x = (torch.randn(T, In, generator=g) * x_scale).to(torch.bfloat16)
+    w = (torch.randn(Out, In, generator=g) * w_scale).to(torch.bfloat16)
+    dy = (torch.randn(T, Out, generator=g) * dy_scale).to(torch.bfloat16)
+    return x, w, dy
+
+
+SMALL = [(1, 16, 16), (77, 48, 80), (128, 128, 256), (200, 272, 400), (333, 256, 528),
+         (130, 1040, 144), (257, 384, 768)]
+
+
+@pytest.mark.parametrize("T,In,Out", SMALL)
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_small_shapes_all_passes(T, In, Out, out_dtype):
+    x, w, dy = _inputs(T, In, Out, seed=T * 7 + In + Out)
+    Q = _passes(x, w, dy)
+    for p in (oracle.FWD, oracle.DGRAD, oracle.WGRAD):
+        _compare_full(p, Q, T, In, Out, out_dtype, "pass %d %s" % (p, (T, In, Out)))
+
+
+def test_format_mixes_and_margins():
+    T, In, Out = 160, 96, 112
+    x, w, dy = _inputs(T, In, Out, seed=5)
+    for fx, fw, fdy in ((E5, E4, E4), (E4, E5, E5), (E5, E5, E5), (E4, E4, E4)):
+        for margins in ((0, 0, 0), (1, 3, 2)):
+            Q = _passes(x, w, dy, margins, fx, fw, fdy)
+            for p in (oracle.FWD, oracle.DGRAD, oracle.WGRAD):
+                _compare_full(p, Q, T, In, Out, torch.float32, "mix %s" % ((fx, fw, fdy),))
+
+
+def test_c0_single_linear_forward_fp32():
+    cfg = workloads.C0
+    x, w, _ = workloads.linear_inputs(0, 0)
+    Q = _passes(x, w, None)
+    lin = cfg.linears[0]
+    _compare_full(oracle.FWD, Q, cfg.tokens, lin.in_features, lin.out_features, torch.float32, "c0")
+
+
+def test_empty_tokens():
+    In, Out = 64, 32
+    z8 = torch.empty((0, In), dtype=torch.uint8, device=DEV)
+    dz8 = torch.empty((0, Out), dtype=torch.uint8, device=DEV)
+    w8 = torch.zeros((Out, In), dtype=torch.uint8, device=DEV)
+    b = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = fp8.fp8_linear_fwd(z8, E4, b, w8, E4, b)
+    assert y.shape == (0, Out)
+    dx = fp8.fp8_linear_bwd_dgrad(dz8, E5, b, w8, E4, b)
+    assert dx.shape == (0, In)
+    dw = torch.full((Out, In), 7.0, dtype=torch.bfloat16, device=DEV)
+    fp8.fp8_linear_bwd_wgrad(dz8, E5, b, z8, E4, b, out=dw)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dw).item() == 0
+
+
+@pytest.mark.parametrize("li", [0, 1, 2])
+def test_c1_gpt111m(li):
+    cfg = workloads.C1
+    lin = cfg.linears[li]
+    x, w, dy = workloads.linear_inputs(1, li)
+    Q = _passes(x, w, dy)
+    for p in (oracle.FWD, oracle.DGRAD, oracle.WGRAD):
+        if li == 0:
+            _compare_full(p, Q, cfg.tokens, lin.in_features, lin.out_features, torch.bfloat16,
+                          "c1 %s pass %d" % (lin.name, p))
+        else:
+            _compare_sampled(p, Q, cfg.tokens, lin.in_features, lin.out_features, torch.bfloat16,
+                             "c1 %s pass %d" % (lin.name, p))
+
+
+@pytest.mark.parametrize("li", [0, 1, 2])
+@pytest.mark.parametrize("margin", [0, 1])
+def test_c2_llama7b_mlp(li, margin):
+    cfg = workloads.C2
+    lin = cfg.linears[li]
+    for step in range(2):                      # bias recomputed on re-drawn tensors each step
+        x, w, dy = workloads.linear_inputs(2, li, step=step)
+        Q = _passes(x, w, dy, (margin, margin, margin))
+        for p in (oracle.FWD, oracle.DGRAD, oracle.WGRAD):
+            _compare_sampled(p, Q, cfg.tokens, lin.in_features, lin.out_features, torch.bfloat16,
+                             "c2 %s m%d s%d pass %d" % (lin.name, margin, step, p),
+                             n_samples=1 << 12, block_cols=512)
+
+
+@pytest.mark.parametrize("li", [0, 1, 2, 3])
+def test_c3_llama70b(li):
+    cfg = workloads.C3
+    lin = cfg.linears[li]
+    x, w, dy = workloads.linear_inputs(3, li)
+    Q = _passes(x, w, dy)
+    for p in (oracle.FWD, oracle.DGRAD, oracle.WGRAD):
+        _compare_sampled(p, Q, cfg.tokens, lin.in_features, lin.out_features, torch.bfloat16,
+                         "c3 %s pass %d" % (lin.name, p), n_samples=1 << 12, block_cols=256)
+
+
+def test_layer_step_matches_oracle():
+    """The whole step object (quantize X, W, dY; fwd, dgrad, wgrad) on c1's first linear."""
+    cfg = workloads.C1
+    lin = cfg.linears[0]
+    x, w, dy = workloads.linear_inputs(1, 0, step=3)
+    layer = fp8.Fp8AmaxLinear(cfg.tokens, lin.in_features, lin.out_features, DEV)
+    y, dx, dw = layer.step(x.to(DEV), w.to(DEV), dy.to(DEV))
+    torch.cuda.synchronize()
+    _, bx, qx = oracle.quantize(x, E4, 0)
+    _, bw, qw = oracle.quantize(w, E4, 0)
+    _, bdy, qdy = oracle.quantize(dy, E5, 0)
+    T, In, Out = cfg.tokens, lin.in_features, lin.out_features
+    qx, qw, qdy = qx.reshape(T, In), qw.reshape(Out, In), qdy.reshape(T, Out)
+    for got, (p, A, fa, ba, B, fb, bb) in zip(
+            (y, dx, dw), ((oracle.FWD, qx, E4, bx, qw, E4, bw), (oracle.DGRAD, qdy, E5, bdy, qw, E4, bw),
+                          (oracle.WGRAD, qdy, E5, bdy, qx, E4, bx))):
+        ref, absref = oracle.linear(p, A, fa, ba, B, fb, bb, T, In, Out)
+        assert_gemm_close(to_f64(got), ref, absref, "layer pass %d" % p)
+
+
+def test_bounded_wait_selftest_and_error_word():
+    assert fp8.fp8_device_error(clear=False) == (0, 0)      # nothing timed out so far
+    assert fp8.fp8_selftest_bounded_wait(50_000_000) == 5   # FP8_ERR_TIMEOUT, then cleared
+    assert fp8.fp8_device_error(clear=False) == (0, 0)
+    # the context is still usable afterwards
+    x = torch.ones(1024, device=DEV)
+    assert fp8.fp8_amax(x).item() == 1.0
