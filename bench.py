@@ -50,7 +50,11 @@ def parse():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="fp8amax", choices=["fp8amax", "reference"])
-    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3"])
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4"],
+                    help="c3: the Llama-2-70B projections (default); c1/c2: smaller layer "
+                         "shapes; c4: the amax+bias+cast sweep alone on one tensor")
+    ap.add_argument("--sweep-log2n", type=int, default=28, help="c4: log2 of the element count")
+    ap.add_argument("--sweep-dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -222,6 +226,48 @@ def run_fp8(args, world, rank, local):
     return res
 
 
+def run_sweep(args, world, rank, local):
+    """amax + bias + cast of one tensor per step (the memory-bound steps alone)."""
+    import fp8_tensor_scaled_b200 as fp8
+    device = torch.device("cuda", local)
+    n = 1 << args.sweep_log2n
+    dt = torch.bfloat16 if args.sweep_dtype == "bf16" else torch.float32
+    x = workloads.sweep_tensor(n, dt, "normal", 1.0, seed=4000, device=device)
+    amax = torch.empty(1, dtype=torch.float32, device=device)
+    bias = torch.empty(1, dtype=torch.int32, device=device)
+    q = torch.empty(n, dtype=torch.uint8, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)     # 2 x L2
+    stream = torch.cuda.current_stream(device)
+    for _ in range(max(3, args.warmup)):
+        fp8.fp8_quantize(x, fp8.E4M3, 0, amax, bias, q)
+    torch.cuda.synchronize(device)
+    tot = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fp8.fp8_quantize(x, fp8.E4M3, 0, amax, bias, q)
+        b.record(stream)
+        b.synchronize()
+        tot += a.elapsed_time(b)
+    ms = max_over_ranks(world, tot / args.steps, device)
+    gbs = (2 * x.element_size() + 1) * n / (ms * 1e-3) / 1e9
+    peaks, src = load_peaks()
+    if rank == 0:
+        print(json.dumps({"metric": "amax+bias+cast GB/s (algorithmic bytes 2*s_in+1)",
+                          "value": round(gbs * world, 1), "unit": "GB/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": max(3, args.warmup),
+                          "ms_per_step": round(ms, 4), "higher_is_better": True,
+                          "scaling": "weak", "dtype": args.sweep_dtype, "data": "synthetic",
+                          "config": {"workload": "amax-bias-cast sweep", "n": n,
+                                     "input": args.sweep_dtype, "l2": "flushed between steps"},
+                          "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
+                                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                       "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None},
+                          "gpu_launches": 2 * args.steps}), flush=True)
+    return 0
+
+
 def run_e2e(args, wl, device, world):
     """Same step through the C ABI from pinned host buffers, copies timed."""
     host_in = [tuple(t.cpu().pin_memory() for t in inp) for inp in wl.inputs]
@@ -256,52 +302,69 @@ def run_e2e(args, wl, device, world):
 
 
 # ------------------------------------------------------------------ CPU oracle
-def oracle_sample(cid, seconds, device_inputs=None):
+def oracle_sample(cid, seconds=15.0):
     """Time the CPU oracle on a bounded sample of one step and extrapolate.
 
-    Sample: for every linear and pass, `r` full output rows of the fp64 oracle
-    matmul, plus amax + bias + cast of the first 2^22 elements of each input
-    tensor.  The whole-step CPU time is extrapolated linearly (the oracle's
-    cost is proportional to output rows and to elements)."""
+    Sample: for every projection and pass, an 8 x `cols` block of output
+    elements of the fp64 oracle matmul (full K each), plus amax + bias + cast of
+    the first 2^22 elements of each of the step's input tensors.  The oracle's
+    cost is linear in output elements x K and in elements cast, so the whole
+    step's CPU time is extrapolated by FLOPs and by elements.  `cols` is sized
+    for roughly `seconds` of CPU time at the oracle's measured rate."""
+    import numpy as np
+
     import oracle
     cfg = workloads.CONFIGS[cid]
+    rng = np.random.default_rng(1)
     g = torch.Generator().manual_seed(1)
     n_q = 1 << 22
     t_quant, n_quant_done, n_quant_total = 0.0, 0, 0
-    t_gemm, f_gemm_done = 0.0, 0
-    rows = 1
-    for li, lin in enumerate(cfg.linears):
-        T, In, Out = cfg.tokens, lin.in_features, lin.out_features
-        # small seeded stand-ins with the real K extents (the oracle's cost does
-        # not depend on the values)
-        for shape in ((T, In), (Out, In), (T, Out)):
+    for lin in cfg.linears:
+        for shape in ((cfg.tokens, lin.in_features), (lin.out_features, lin.in_features),
+                      (cfg.tokens, lin.out_features)):
             n_quant_total += shape[0] * shape[1]
             x = torch.randn(min(n_q, shape[0] * shape[1]), generator=g).to(torch.bfloat16)
             t0 = time.perf_counter()
             oracle.quantize(x, 0, 0)
             t_quant += time.perf_counter() - t0
             n_quant_done += x.numel()
-        xq = torch.randint(0, 120, (rows, In), generator=g, dtype=torch.uint8).numpy()
-        wq = torch.randint(0, 120, (Out, In), generator=g, dtype=torch.uint8).numpy()
-        dq = torch.randint(0, 120, (T, Out), generator=g, dtype=torch.uint8).numpy()
-        xfull = torch.randint(0, 120, (T, In), generator=g, dtype=torch.uint8).numpy()
-        # fwd rows: Y[r, :] needs X[r, :] and all of W
-        t0 = time.perf_counter()
-        oracle.linear(oracle.FWD, xq, 0, 0, wq, 0, 0, rows, In, Out, with_abs=False)
-        # dgrad rows: dX[r, :] needs dY[r, :] and all of W
-        oracle.linear(oracle.DGRAD, dq[:rows], 1, 0, wq, 0, 0, rows, In, Out, with_abs=False)
-        # wgrad rows: dW[o, :] for o < rows needs dY[:, o] and all of X
-        oracle.linear(oracle.WGRAD, dq[:, :16].copy(), 1, 0, xfull, 0, 0, T, In, 16,
-                      with_abs=False)
-        t_gemm += time.perf_counter() - t0
-        f_gemm_done += 2 * rows * In * Out + 2 * rows * Out * In + 2 * 16 * T * In
+
+    def block(rows, cols):
+        r, c = np.meshgrid(np.arange(rows), np.arange(cols), indexing="ij")
+        return r.ravel(), c.ravel()
+
+    # measure the rate on a small block first, then size the sample to `seconds`
+    T = cfg.tokens
+    lin0 = cfg.linears[0]
+    X = rng.integers(0, 120, (T, lin0.in_features), dtype=np.uint8)
+    W = rng.integers(0, 120, (lin0.out_features, lin0.in_features), dtype=np.uint8)
+    r, c = block(8, 64)
+    t0 = time.perf_counter()
+    oracle.linear_entries(oracle.FWD, X, 0, 0, W, 0, 0, T, lin0.in_features, lin0.out_features,
+                          r, c)
+    rate = 2.0 * r.size * lin0.in_features / (time.perf_counter() - t0)       # FLOP/s
+    k_sum = sum(l.in_features + l.out_features + T for l in cfg.linears)
+    cols = int(max(16, min(4096, seconds * rate / (2.0 * 8 * k_sum))))
+
+    t_gemm, f_gemm_done = 0.0, 0
+    for lin in cfg.linears:
+        In, Out = lin.in_features, lin.out_features
+        X = rng.integers(0, 120, (T, In), dtype=np.uint8)
+        W = rng.integers(0, 120, (Out, In), dtype=np.uint8)
+        dY = rng.integers(0, 120, (T, Out), dtype=np.uint8)
+        for p, A, fa, B, K, ncols in ((oracle.FWD, X, 0, W, In, Out), (oracle.DGRAD, dY, 1, W, Out, In),
+                                      (oracle.WGRAD, dY, 1, X, T, In)):
+            r, c = block(8, min(cols, ncols))
+            t0 = time.perf_counter()
+            oracle.linear_entries(p, A, fa, 0, B, 0, 0, T, In, Out, r, c)
+            t_gemm += time.perf_counter() - t0
+            f_gemm_done += 2 * r.size * K
     flops = cfg.flops_per_step()
-    est_gemm = t_gemm * flops / f_gemm_done
-    est_quant = t_quant * n_quant_total / n_quant_done
-    est_step = est_gemm + est_quant
-    sample = ("oracle on 1 output row of fwd and dgrad and 16 rows of wgrad per projection "
-              "(full K), plus amax+bias+cast of 2^22 elements of each of the 12 input tensors; "
-              "whole-step time extrapolated by FLOPs and by elements")
+    est_step = t_gemm * flops / f_gemm_done + t_quant * n_quant_total / n_quant_done
+    sample = ("CPU oracle on an 8 x %d block of output elements (full K) of each of the %d "
+              "matmuls of the step, plus amax+bias+cast of 2^22 elements of each of the %d "
+              "input tensors; whole-step time extrapolated by FLOPs and elements"
+              % (cols, 3 * len(cfg.linears), 3 * len(cfg.linears)))
     return {"value": flops / est_step / 1e12, "unit": UNIT, "cores": oracle.num_threads(),
             "kind": "oracle", "sample": sample, "sample_seconds": round(t_gemm + t_quant, 3),
             "est_step_seconds": round(est_step, 1)}
@@ -356,6 +419,12 @@ def main():
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}))
         return 1
+    if args.workload == "c4":
+        rc = run_sweep(args, world, rank, local)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
     peaks, peak_src = load_peaks()
     r = run_fp8(args, world, rank, local)
     wl = r["wl"]
