@@ -82,18 +82,35 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
-constexpr int BM = 128;                 // UMMA M (one CTA)
+// Tile shapes.  kCta = 1: one CTA computes a 128 x 256 tile with
+// tcgen05.mma.cta_group::1 (M=128, N=256).  kCta = 2: a pair of CTAs (a
+// cluster of 2) computes a 256 x 256 tile with cta_group::2 (M=256, N=256):
+// CTA r loads rows [128r, 128r+128) of the A tile and of the B tile into its
+// own shared memory and holds rows [128r, 128r+128) of the accumulator in its
+// own tensor memory; the leader (r = 0) issues the MMAs for both.
 constexpr int BN = 256;                 // UMMA N
 constexpr int BK = 128;                 // K per stage: one 128-byte swizzle row of FP8
 constexpr int UK = 32;                  // K per tcgen05.mma of kind::f8f6f4
-constexpr int STAGES = 4;
-constexpr uint32_t A_BYTES = BM * BK;   // 16 KB
-constexpr uint32_t B_BYTES = BN * BK;   // 32 KB
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t A_BYTES = 128 * BK;  // 16 KB: 128 rows of A per CTA
 constexpr uint32_t TMEM_COLS = 512;     // 2 accumulators x 256 fp32 columns
 constexpr int kThreads = 192;           // 6 warps
-constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1;
-constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + kNumBars * 8 + 16;
+
+template <int kCta> struct Cfg;
+template <> struct Cfg<1> {
+  static constexpr int BM = 128;                       // rows per tile
+  static constexpr uint32_t B_BYTES = BN * BK;         // 32 KB: all 256 B rows
+  static constexpr int STAGES = 4;
+};
+template <> struct Cfg<2> {
+  static constexpr int BM = 256;
+  static constexpr uint32_t B_BYTES = (BN / 2) * BK;   // 16 KB: this CTA's 128 B rows
+  static constexpr int STAGES = 6;
+};
+template <int kCta> constexpr uint32_t stage_bytes() { return A_BYTES + Cfg<kCta>::B_BYTES; }
+template <int kCta> constexpr int num_bars() { return 2 * Cfg<kCta>::STAGES + 2 + 2 + 1; }
+template <int kCta> constexpr size_t smem_bytes() {
+  return 1024 + Cfg<kCta>::STAGES * stage_bytes<kCta>() + num_bars<kCta>() * 8 + 16;
+}
 
 struct Params {
   int M, N, K;
@@ -146,10 +163,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-template <bool kAMN, bool kBMN, bool kOutF32>
+template <int kCta>
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         int site, uint64_t limit_ns) {
+  if (kCta == 1) return mbar_wait_bounded(bar, parity, abort_flag, site, limit_ns);
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      *abort_flag = 1;
+      record_device_error(site);
+      return false;
+    }
+  }
+}
+
+template <int kCta, bool kAMN, bool kBMN, bool kOutF32>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b, const Params p) {
+  using C = Cfg<kCta>;
+  constexpr int STAGES = C::STAGES;
+  constexpr uint32_t B_BYTES = C::B_BYTES;
+  constexpr uint32_t STAGE_BYTES = stage_bytes<kCta>();
+  constexpr int kNumBars = num_bars<kCta>();
+
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -168,15 +210,19 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
+  const uint32_t rank = kCta == 2 ? cluster_ctarank() : 0u;     // 0 = leader
+  const bool leader = rank == 0;
+  const int unit = kCta == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int num_units = kCta == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(full_bar(s), 1);            // the leader's producer arrives (with expect_tx)
+      mbar_init(empty_bar(s), 1);           // one tcgen05.commit per stage use
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 4);          // one arrival per epilogue warp
+      mbar_init(tempty_bar(a), 4 * kCta);   // one arrival per epilogue warp of the pair
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -185,71 +231,93 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     tma_prefetch_desc(&tmap_b);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    if (kCta == 2) {
+      tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (kCta == 2) cluster_sync();            // both CTAs' barriers and TMEM ready
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
     // ----------------------------- TMA producer -----------------------------
+    // Both CTAs load their own halves; the copies complete on the leader's
+    // full barrier, which the leader arms with the bytes of both CTAs.
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t armed_mask = 0, armed_parity = 0;   // per stage: last armed phase
-    for (int t = blockIdx.x; t < p.num_tiles && !*abort_flag; t += gridDim.x) {
+    uint32_t armed_mask = 0, armed_parity = 0;   // leader: last armed phase per stage
+    for (int t = unit; t < p.num_tiles && !*abort_flag; t += num_units) {
       int mb, nb;
       tile_coords(t, p, mb, nb);
+      const int a_row = mb * C::BM + static_cast<int>(rank) * 128;
+      const int b_row = nb * BN + (kCta == 2 ? static_cast<int>(rank) * 128 : 0);
       bool ok = true;
       for (int kb = 0; kb < p.num_k_blocks; ++kb) {
-        if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, kSiteProducerEmpty,
-                               p.wait_limit_ns)) {
+        if (!wait_bar<kCta>(empty_bar(stage), phase ^ 1u, abort_flag, kSiteProducerEmpty,
+                            p.wait_limit_ns)) {
           ok = false;
           break;
         }
         const uint32_t fb = full_bar(stage);
-        mbar_arrive_expect_tx(fb, STAGE_BYTES);
-        armed_mask |= 1u << stage;
-        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        if (leader) {
+          mbar_arrive_expect_tx(fb, kCta * STAGE_BYTES);
+          armed_mask |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        }
         const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
         const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
         const int k0 = kb * BK;
-        if (kAMN) tma_load_2d(a_dst, &tmap_a, fb, mb * BM, k0);
-        else      tma_load_2d(a_dst, &tmap_a, fb, k0, mb * BM);
-        if (kBMN) {
-          tma_load_2d(b_dst, &tmap_b, fb, nb * BN, k0);
-          tma_load_2d(b_dst + BK * 128, &tmap_b, fb, nb * BN + 128, k0);
+        if (kCta == 2) {
+          const uint32_t fb_leader = mapa_shared(fb, 0);
+          if (kAMN) tma_load_2d_pair(a_dst, &tmap_a, fb_leader, a_row, k0);
+          else      tma_load_2d_pair(a_dst, &tmap_a, fb_leader, k0, a_row);
+          if (kBMN) tma_load_2d_pair(b_dst, &tmap_b, fb_leader, b_row, k0);
+          else      tma_load_2d_pair(b_dst, &tmap_b, fb_leader, k0, b_row);
         } else {
-          tma_load_2d(b_dst, &tmap_b, fb, k0, nb * BN);
+          if (kAMN) tma_load_2d(a_dst, &tmap_a, fb, a_row, k0);
+          else      tma_load_2d(a_dst, &tmap_a, fb, k0, a_row);
+          if (kBMN) {
+            tma_load_2d(b_dst, &tmap_b, fb, b_row, k0);
+            tma_load_2d(b_dst + BK * 128, &tmap_b, fb, b_row + 128, k0);
+          } else {
+            tma_load_2d(b_dst, &tmap_b, fb, k0, b_row);
+          }
         }
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
     }
-    // Every copy this thread issued completes its stage's full barrier; wait
-    // for the last one of each stage so that no copy is still landing in shared
-    // memory when the block exits (immediate in the normal case).
+    // Every copy the leader armed completes its stage's full barrier; wait for
+    // the last one of each stage so that no copy is still landing when the
+    // block exits (immediate in the normal case; the pair's final cluster
+    // barrier covers the peer's copies, which count on the same barriers).
     int never = 0;
-    for (int s = 0; s < STAGES; ++s)
-      if (armed_mask & (1u << s))
-        mbar_wait_bounded(full_bar(s), (armed_parity >> s) & 1u, &never, kSiteDrain, kDrainLimitNs);
-  } else if (warp == 1 && lane == 0) {
+    if (leader)
+      for (int s = 0; s < STAGES; ++s)
+        if (armed_mask & (1u << s))
+          wait_bar<kCta>(full_bar(s), (armed_parity >> s) & 1u, &never, kSiteDrain, kDrainLimitNs);
+  } else if (warp == 1 && lane == 0 && leader) {
     // ------------------------------ MMA issuer ------------------------------
     int stage = 0;
     uint32_t phase = 0;
     int local = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+    for (int t = unit; t < p.num_tiles; t += num_units, ++local) {
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
-      if (!mbar_wait_bounded(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, kSiteMmaTmemEmpty,
-                             p.wait_limit_ns))
+      if (!wait_bar<kCta>(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, kSiteMmaTmemEmpty,
+                          p.wait_limit_ns))
         break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
       bool ok = true;
       for (int kb = 0; kb < p.num_k_blocks; ++kb) {
-        if (!mbar_wait_bounded(full_bar(stage), phase, abort_flag, kSiteMmaFull, p.wait_limit_ns)) {
+        if (!wait_bar<kCta>(full_bar(stage), phase, abort_flag, kSiteMmaFull, p.wait_limit_ns)) {
           ok = false;
           break;
         }
@@ -258,38 +326,45 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const uint32_t b_base = smem_u32(sB + stage * B_BYTES);
 #pragma unroll
         for (int k = 0; k < BK / UK; ++k) {
-          mma_f8f6f4(d_tmem, operand_desc<kAMN>(a_base, k), operand_desc<kBMN>(b_base, k), p.idesc,
-                     (kb | k) != 0 ? 1u : 0u);
+          const uint64_t ad = operand_desc<kAMN>(a_base, k);
+          const uint64_t bd = operand_desc<kBMN>(b_base, k);
+          if (kCta == 2) mma_f8f6f4_pair(d_tmem, ad, bd, p.idesc, (kb | k) != 0 ? 1u : 0u);
+          else           mma_f8f6f4(d_tmem, ad, bd, p.idesc, (kb | k) != 0 ? 1u : 0u);
         }
-        mma_commit(empty_bar(stage));     // frees the stage once these MMAs have read it
+        // frees the stage (in both CTAs) once these MMAs have read it
+        if (kCta == 2) mma_commit_pair_mc(empty_bar(stage), 0x3);
+        else           mma_commit(empty_bar(stage));
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
-      mma_commit(tfull_bar(acc));         // accumulator complete
+      // accumulator complete (in both CTAs)
+      if (kCta == 2) mma_commit_pair_mc(tfull_bar(acc), 0x3);
+      else           mma_commit(tfull_bar(acc));
     }
     // Drain: the commit arrives only after every MMA this thread issued is done.
-    mma_commit(drain_bar);
+    if (kCta == 2) mma_commit_pair_mc(drain_bar, 0x1);
+    else           mma_commit(drain_bar);
     int never = 0;
-    mbar_wait_bounded(drain_bar, 0, &never, kSiteDrain, kDrainLimitNs);
+    wait_bar<kCta>(drain_bar, 0, &never, kSiteDrain, kDrainLimitNs);
   } else if (warp >= 2) {
     // ------------------------------- epilogue -------------------------------
     const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
-    const int row_in_tile = quarter * 32 + lane;
+    const int row_in_tile = static_cast<int>(rank) * 128 + quarter * 32 + lane;
     const Pow2Scale sc = make_pow2_scale(-(*p.bias_a + *p.bias_b));
     int local = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+    for (int t = unit; t < p.num_tiles; t += num_units, ++local) {
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       int ok = 1;
       if (lane == 0)
-        ok = mbar_wait_bounded(tfull_bar(acc), use & 1u, abort_flag, kSiteEpilogueTmemFull,
-                               p.wait_limit_ns) ? 1 : 0;
+        ok = wait_bar<kCta>(tfull_bar(acc), use & 1u, abort_flag, kSiteEpilogueTmemFull,
+                            p.wait_limit_ns) ? 1 : 0;
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       tc_fence_after();
       int mb, nb;
       tile_coords(t, p, mb, nb);
-      const int64_t row = static_cast<int64_t>(mb) * BM + row_in_tile;
+      const int64_t row = static_cast<int64_t>(mb) * C::BM + row_in_tile;
       const bool row_ok = row < p.M;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
@@ -335,15 +410,24 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (lane == 0) {
+        if (kCta == 2) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));  // leader's barrier
+        else           mbar_arrive(tempty_bar(acc));
+      }
     }
   }
 
+  // Teardown: every role has left its loop (all waits are bounded).  The pair
+  // meets once more so that no CTA exits or frees its tensor memory while the
+  // other can still reach its shared memory or tensor memory.
   __syncthreads();
+  __syncwarp();
+  tc_fence_before();
+  if (kCta == 2) cluster_sync();
+  tc_fence_after();
   if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (kCta == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else           tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -409,12 +493,18 @@ int sm_count() {
   return g_sm_count[dev];
 }
 
-template <bool kAMN, bool kBMN, bool kOutF32>
+template <int kCta, bool kAMN, bool kBMN, bool kOutF32>
 int launch_t(const GemmArgs& g, cudaStream_t s) {
+  constexpr int BM = Cfg<kCta>::BM;
+  constexpr size_t kSmem = smem_bytes<kCta>();
+  // TMA boxes: 128 x 128 bytes for A (this CTA's rows) and, for B, all 256
+  // rows (one CTA, K-major) or 128 rows / MN columns (MN-major, or a pair).
+  const uint32_t b_box_rows = (kCta == 1 && !kBMN) ? BN : 128;
   CUtensorMap ta, tb;
   const uint64_t M = g.M, N = g.N, K = g.K;
-  const bool ok_a = kAMN ? encode_2d(&ta, g.a, M, K, 128, BK) : encode_2d(&ta, g.a, K, M, BK, BM);
-  const bool ok_b = kBMN ? encode_2d(&tb, g.b, N, K, 128, BK) : encode_2d(&tb, g.b, K, N, BK, BN);
+  const bool ok_a = kAMN ? encode_2d(&ta, g.a, M, K, 128, BK) : encode_2d(&ta, g.a, K, M, BK, 128);
+  const bool ok_b = kBMN ? encode_2d(&tb, g.b, N, K, 128, BK)
+                         : encode_2d(&tb, g.b, K, N, BK, b_box_rows);
   if (!ok_a || !ok_b) return FP8_ERR_CUDA;
 
   Params p;
@@ -432,42 +522,74 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
             | (static_cast<uint32_t>(kAMN) << 15)         // A major: 0 K, 1 MN
             | (static_cast<uint32_t>(kBMN) << 16)         // B major
             | (static_cast<uint32_t>(BN >> 3) << 17)      // N / 8
-            | (static_cast<uint32_t>(BM >> 4) << 24);     // M / 16
+            | (static_cast<uint32_t>(BM >> 4) << 24);     // M / 16 (256 for a pair)
   p.bias_a = g.bias_a;
   p.bias_b = g.bias_b;
   p.d = g.d;
   p.wait_limit_ns = kWaitLimitNs;
 
-  static bool attr_set[64];
+  static int max_units[64];      // co-resident CTAs (1-CTA) or clusters (pair), per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  auto kern = fp8_gemm_kernel<kAMN, kBMN, kOutF32>;
-  if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess)
-      return FP8_ERR_CUDA;
-    attr_set[dev] = true;
+  auto kern = fp8_gemm_kernel<kCta, kAMN, kBMN, kOutF32>;
+
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmem;
+  cfg.stream = s;
+  if (kCta == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
   }
-  const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
-  kern<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, p);
+  if (max_units[dev] == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmem)) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    int units = sm_count();
+    if (kCta == 2) {
+      int clusters = 0;
+      cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess || clusters < 1) {
+        cudaGetLastError();
+        clusters = sm_count() / 2;
+      }
+      units = clusters;
+    }
+    max_units[dev] = units;
+  }
+  const int units = p.num_tiles < max_units[dev] ? p.num_tiles : max_units[dev];
+  cfg.gridDim = dim3(static_cast<unsigned>(units * kCta), 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return FP8_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+template <bool kAMN, bool kBMN, bool kOutF32>
+int launch_pick(const GemmArgs& g, cudaStream_t s) {
+  // One 128-row tile covers M: a single CTA per tile; otherwise CTA pairs.
+  if (g.M <= 128) return launch_t<1, kAMN, kBMN, kOutF32>(g, s);
+  return launch_t<2, kAMN, kBMN, kOutF32>(g, s);
 }
 
 }  // namespace
 
 int launch_gemm(const GemmArgs& g, cudaStream_t s) {
   // limits of the 32-bit tile arithmetic and of the TMA tensor map
-  if (g.M > (1LL << 31) - 1 - BM || g.N > (1LL << 31) - 1 - BN || g.K > (1LL << 31) - 1 - BK)
+  if (g.M > (1LL << 31) - 1 - 256 || g.N > (1LL << 31) - 1 - BN || g.K > (1LL << 31) - 1 - BK)
     return FP8_ERR_UNSUPPORTED;
   const int key = (g.a_mn_major ? 4 : 0) | (g.b_mn_major ? 2 : 0) | (g.d_fp32 ? 1 : 0);
   switch (key) {
-    case 0: return launch_t<false, false, false>(g, s);
-    case 1: return launch_t<false, false, true>(g, s);
-    case 2: return launch_t<false, true, false>(g, s);
-    case 3: return launch_t<false, true, true>(g, s);
-    case 6: return launch_t<true, true, false>(g, s);
-    case 7: return launch_t<true, true, true>(g, s);
+    case 0: return launch_pick<false, false, false>(g, s);
+    case 1: return launch_pick<false, false, true>(g, s);
+    case 2: return launch_pick<false, true, false>(g, s);
+    case 3: return launch_pick<false, true, true>(g, s);
+    case 6: return launch_pick<true, true, false>(g, s);
+    case 7: return launch_pick<true, true, true>(g, s);
     default: return FP8_ERR_UNSUPPORTED;   // MN-major A with K-major B: no pass uses it
   }
 }
