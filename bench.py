@@ -58,9 +58,36 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="run each projection's quantization and GEMMs strictly in order")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="approximate CPU time of the oracle sample")
     return ap.parse_args()
+
+
+def gemm_traffic_per_launch():
+    """DRAM bytes per GEMM launch of the step, from the committed ncu summary,
+    or None when the GEMM sources changed since those counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "fp8_gemm_llama2_70b_traffic.md")
+    if not os.path.exists(path):
+        return None
+    h = hashlib.sha256()
+    for f in ("gemm_sm100.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "fp8_tensor_scaled_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    fields = {}
+    with open(path) as fh:
+        for line in fh:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    if fields.get("source-sha256") != h.hexdigest():
+        return None
+    try:
+        return int(fields["dram-bytes-per-launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 def load_peaks():
@@ -155,9 +182,9 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the step
 class Workload:
-    def __init__(self, cid, device, seed_step=0):
+    def __init__(self, cid, device, seed_step=0, overlap=True):
         import fp8_tensor_scaled_b200 as fp8
-        self.fp8 = fp8
+        from fp8_tensor_scaled_b200.layer import Fp8AmaxStep
         self.cfg = workloads.CONFIGS[cid]
         self.device = device
         self.inputs, self.layers = [], []
@@ -168,36 +195,33 @@ class Workload:
             self.layers.append(fp8.Fp8AmaxLinear(self.cfg.tokens, lin.in_features,
                                                  lin.out_features, device, self.cfg.out_dtype,
                                                  m, m, m))
-        self.flops = sum(l.flops() for l in self.layers)
+        self.stepper = Fp8AmaxStep(self.layers, overlap=overlap)
+        self.flops = self.stepper.flops()
         # algorithmic bytes of amax + cast: read the input twice, write one FP8 byte
         self.quant_bytes = sum((2 * t.element_size() + 1) * t.numel()
                                for inp in self.inputs for t in inp)
         self.kernels_per_step = len(self.layers) * (3 * 2 + 3)   # 3 x (amax + cast) + 3 GEMMs
 
-    def step(self, ev=None):
-        for i, (layer, (x, w, dy)) in enumerate(zip(self.layers, self.inputs)):
-            if ev is not None:
-                ev[i][0].record()
-            layer.quantize(x, w, dy)
-            if ev is not None:
-                ev[i][1].record()
-            layer.gemms()
-            if ev is not None:
-                ev[i][2].record()
+    def new_timing(self):
+        n = len(self.layers)
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        return {"q": [[ev(), ev()] for _ in range(n)], "g": [[ev(), ev()] for _ in range(n)]}
+
+    def step(self, timing=None):
+        self.stepper.step(self.inputs, timing=timing)
 
 
 def run_fp8(args, world, rank, local):
     device = torch.device("cuda", local)
     cid = int(args.workload[1:])
-    wl = Workload(cid, device)
+    wl = Workload(cid, device, overlap=not args.no_overlap)
     stream = torch.cuda.current_stream(device)
     for _ in range(max(3, args.warmup)):
         wl.step()
     torch.cuda.synchronize(device)
 
     nlin = len(wl.layers)
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nlin)]
-           for _ in range(args.steps)]
+    timings = [wl.new_timing() for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(device)
@@ -205,19 +229,17 @@ def run_fp8(args, world, rank, local):
     time.sleep(0.3)
     start.record(stream)
     for s in range(args.steps):
-        wl.step(evs[s])
+        wl.step(timings[s])
     end.record(stream)
     torch.cuda.synchronize(device)
     clocks = sampler.stop()
     barrier(world)
     ms_local = start.elapsed_time(end)
     ms = max_over_ranks(world, ms_local, device)
-    quant_ms = sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps)
-                   for i in range(nlin))
-    gemm_ms = sum(evs[s][i][1].elapsed_time(evs[s][i][2]) for s in range(args.steps)
-                  for i in range(nlin))
-    per_linear_gemm_ms = [sum(evs[s][i][1].elapsed_time(evs[s][i][2])
-                              for s in range(args.steps)) / args.steps for i in range(nlin)]
+    span = lambda pair: pair[0].elapsed_time(pair[1])
+    quant_ms = sum(span(t["q"][i]) for t in timings for i in range(nlin))
+    gemm_ms = sum(span(t["g"][i]) for t in timings for i in range(nlin))
+    per_linear_gemm_ms = [sum(span(t["g"][i]) for t in timings) / args.steps for i in range(nlin)]
     res = dict(ms=ms, ms_local=ms_local, quant_ms=quant_ms, gemm_ms=gemm_ms,
                per_linear_gemm_ms=per_linear_gemm_ms, clocks=clocks, wl=wl)
 
@@ -269,7 +291,9 @@ def run_sweep(args, world, rank, local):
 
 
 def run_e2e(args, wl, device, world):
-    """Same step through the C ABI from pinned host buffers, copies timed."""
+    """Same step through the C ABI from pinned HOST buffers: every step copies
+    X, W, dY of each projection in and its Y, dX, dW out (copy streams in both
+    directions overlap each other and the compute), all inside the timed region."""
     host_in = [tuple(t.cpu().pin_memory() for t in inp) for inp in wl.inputs]
     host_out = [tuple(torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
                       for o in (l.y, l.dx, l.dw)) for l in wl.layers]
@@ -278,15 +302,7 @@ def run_e2e(args, wl, device, world):
     stream = torch.cuda.current_stream(device)
 
     def one():
-        for (hx, hw, hdy), (x, w, dy) in zip(host_in, wl.inputs):
-            x.copy_(hx, non_blocking=True)
-            w.copy_(hw, non_blocking=True)
-            dy.copy_(hdy, non_blocking=True)
-        wl.step()
-        for layer, (hy, hdx, hdw) in zip(wl.layers, host_out):
-            hy.copy_(layer.y, non_blocking=True)
-            hdx.copy_(layer.dx, non_blocking=True)
-            hdw.copy_(layer.dw, non_blocking=True)
+        wl.stepper.step_from_host(host_in, wl.inputs, host_out)
 
     one()
     torch.cuda.synchronize(device)
@@ -434,20 +450,30 @@ def main():
     value = total_flops / (ms_step * 1e-3) / 1e12
     gemm_tflops = wl.flops * steps / (r["gemm_ms"] * 1e-3) / 1e12
     quant_gbs = wl.quant_bytes * steps / (r["quant_ms"] * 1e-3) / 1e9
-    fp8_peak = peaks["bf16_tflops_sustained"] * NOMINAL_FP8_OVER_BF16
+    # Dense FP8 peak: the measured BF16 cuBLAS rate x the nominal FP8/BF16 ratio.
+    # The burst figure is the denominator (the timed region is well under the
+    # seconds-long loop of the sustained figure, and its clocks are recorded in
+    # `clocks`); the sustained-derived figure is reported beside it.
+    fp8_peak = peaks["bf16_tflops"] * NOMINAL_FP8_OVER_BF16
+    fp8_peak_sus = peaks["bf16_tflops_sustained"] * NOMINAL_FP8_OVER_BF16
     hbm_peak = peaks["hbm_gbs"]
+    traffic = gemm_traffic_per_launch()
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8",
         "data": "synthetic", "config": config_dict(wl.cfg, world),
         "gemm_tflops": round(gemm_tflops, 2), "quant_gbs": round(quant_gbs, 1),
+        "overlap": not args.no_overlap,
         "per_linear_gemm_ms": [round(x, 4) for x in r["per_linear_gemm_ms"]],
         "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 2), "peak": round(fp8_peak, 1),
-                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp8_peak, 4), "traffic": None,
-                     "kernel": "fp8_gemm_kernel (fwd/dgrad/wgrad)",
-                     "peak_source": "%s bf16 sustained x %.0f (dense FP8/BF16 ratio)"
-                                    % (peak_src, NOMINAL_FP8_OVER_BF16)},
+                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp8_peak, 4),
+                     "traffic": traffic if args.workload == "c3" else None,
+                     "kernel": "fp8_gemm_kernel (fwd/dgrad/wgrad, all 12 launches of a step)",
+                     "peak_source": "%s bf16 burst x %.0f (dense FP8/BF16 ratio)"
+                                    % (peak_src, NOMINAL_FP8_OVER_BF16),
+                     "frac_of_sustained_peak": round(gemm_tflops / fp8_peak_sus, 4),
+                     "frac_of_nominal_4500": round(gemm_tflops / 4500.0, 4)},
         "roofline_quant": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm_peak,
                            "unit": "GB/s", "frac": round(quant_gbs / hbm_peak, 4),
                            "kernel": "amax_kernel + cast_kernel",
