@@ -58,6 +58,10 @@ def lib():
         "fp8_linear_fwd": [vp, c.c_int, vp, vp, c.c_int, vp, i64, i64, i64, vp, c.c_int, vp],
         "fp8_linear_bwd_dgrad": [vp, c.c_int, vp, vp, c.c_int, vp, i64, i64, i64, vp, c.c_int, vp],
         "fp8_linear_bwd_wgrad": [vp, c.c_int, vp, vp, c.c_int, vp, i64, i64, i64, vp, c.c_int, vp],
+        "fp8_linear_fwd_amax": [vp, c.c_int, vp, vp, c.c_int, vp, i64, i64, i64, vp, c.c_int, vp,
+                                vp],
+        "fp8_linear_bwd_dgrad_amax": [vp, c.c_int, vp, vp, c.c_int, vp, i64, i64, i64, vp, c.c_int,
+                                      vp, vp],
         "fp8_device_error": [c.c_int, vp],
         "fp8_selftest_bounded_wait": [u64],
         "fp8_abi_version": [],
@@ -165,35 +169,50 @@ def fp8_quantize(x: torch.Tensor, fmt: int, margin: int = 0, amax: torch.Tensor 
 _OUT = {torch.bfloat16: BF16, torch.float32: FP32}
 
 
-def _linear(name, a, fa, ba, b, fb, bb, T, in_, out_, shape, out, out_dtype):
+def _linear(name, a, fa, ba, b, fb, bb, T, in_, out_, shape, out, out_dtype, amax=False):
     _need_cuda(a, ba, b, bb, out)
     dev = ba.device
     if out is None:
         out = torch.empty(shape, dtype=out_dtype, device=dev)
     if tuple(out.shape) != tuple(shape) or out.dtype not in _OUT:
         raise ValueError("output must be %s of bfloat16/float32" % (shape,))
+    args = [_ptr(a), int(fa), _ptr(ba), _ptr(b), int(fb), _ptr(bb), int(T), int(in_), int(out_),
+            _ptr(out), _OUT[out.dtype]]
+    if amax is not False:
+        if amax is None or amax is True:
+            amax = torch.empty(1, dtype=torch.float32, device=dev)
+        _need_cuda(amax)
+        name = name + "_amax"
+        args.append(_ptr(amax))
     f = getattr(lib(), name)
-    _check(name, f(_ptr(a), int(fa), _ptr(ba), _ptr(b), int(fb), _ptr(bb), int(T), int(in_),
-                   int(out_), _ptr(out), _OUT[out.dtype], ctypes.c_void_p(_stream_ptr(ba))))
-    return out
+    _check(name, f(*args, ctypes.c_void_p(_stream_ptr(ba))))
+    return out if amax is False else (out, amax)
 
 
-def fp8_linear_fwd(x8, fx, bias_x, w8, fw, bias_w, out=None, out_dtype=torch.bfloat16):
-    """Y [T,out] = (X8 [T,in] . W8 [out,in]^T) * 2^-(bias_x + bias_w)."""
+def fp8_linear_fwd(x8, fx, bias_x, w8, fw, bias_w, out=None, out_dtype=torch.bfloat16,
+                   amax=False):
+    """Y [T,out] = (X8 [T,in] . W8 [out,in]^T) * 2^-(bias_x + bias_w).
+
+    amax=True (or a float32 [1] device tensor) calls fp8_linear_fwd_amax and
+    returns (Y, max|Y|) with the amax taken in the GEMM epilogue."""
     T, in_ = x8.shape
     out_ = w8.shape[0]
     assert w8.shape[1] == in_
     return _linear("fp8_linear_fwd", x8, fx, bias_x, w8, fw, bias_w, T, in_, out_, (T, out_),
-                   out, out_dtype)
+                   out, out_dtype, amax)
 
 
-def fp8_linear_bwd_dgrad(dy8, fdy, bias_dy, w8, fw, bias_w, out=None, out_dtype=torch.bfloat16):
-    """dX [T,in] = (dY8 [T,out] . W8 [out,in]) * 2^-(bias_dy + bias_w)."""
+def fp8_linear_bwd_dgrad(dy8, fdy, bias_dy, w8, fw, bias_w, out=None, out_dtype=torch.bfloat16,
+                         amax=False):
+    """dX [T,in] = (dY8 [T,out] . W8 [out,in]) * 2^-(bias_dy + bias_w).
+
+    amax=True (or a float32 [1] device tensor) calls fp8_linear_bwd_dgrad_amax
+    and returns (dX, max|dX|)."""
     T, out_ = dy8.shape
     in_ = w8.shape[1]
     assert w8.shape[0] == out_
     return _linear("fp8_linear_bwd_dgrad", dy8, fdy, bias_dy, w8, fw, bias_w, T, in_, out_,
-                   (T, in_), out, out_dtype)
+                   (T, in_), out, out_dtype, amax)
 
 
 def fp8_linear_bwd_wgrad(dy8, fdy, bias_dy, x8, fx, bias_x, out=None, out_dtype=torch.bfloat16):

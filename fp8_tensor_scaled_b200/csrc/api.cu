@@ -67,7 +67,7 @@ fp8_status_t check_linear(const uint8_t* a, bool a_tok, int fa, const int32_t* b
 
 fp8_status_t run_gemm(const uint8_t* a, int fa, bool a_mn, const int32_t* ba, const uint8_t* b,
                       int fb, bool b_mn, const int32_t* bb, int64_t M, int64_t N, int64_t K,
-                      void* d, int ddt, cudaStream_t s) {
+                      void* d, int ddt, cudaStream_t s, float* d_amax = nullptr) {
   GemmArgs g;
   g.a = a;
   g.b = b;
@@ -79,6 +79,7 @@ fp8_status_t run_gemm(const uint8_t* a, int fa, bool a_mn, const int32_t* ba, co
   g.bias_b = bb;
   g.d = d;
   g.d_fp32 = ddt == FP8_DTYPE_FP32;
+  g.d_amax = d_amax;
   g.M = M;
   g.N = N;
   g.K = K;
@@ -185,6 +186,41 @@ fp8_status_t fp8_linear_bwd_wgrad(const uint8_t* dy8, fp8_format_t fdy, const in
   }
   return run_gemm(dy8, fdy, true, bias_dy, x8, fx, true, bias_x, out, in, T, dw, dw_dtype,
                   as_stream(stream));
+}
+
+fp8_status_t fp8_linear_fwd_amax(const uint8_t* x8, fp8_format_t fx, const int32_t* bias_x,
+                                 const uint8_t* w8, fp8_format_t fw, const int32_t* bias_w,
+                                 int64_t T, int64_t in, int64_t out, void* y, fp8_dtype_t y_dtype,
+                                 float* y_amax, void* stream) {
+  if (!y_amax) return FP8_ERR_INVALID_ARGUMENT;
+  if (reinterpret_cast<uintptr_t>(y_amax) & 3u) return FP8_ERR_MISALIGNED;
+  if (fp8_status_t st = check_linear(x8, true, fx, bias_x, w8, false, fw, bias_w, T, in, out, y,
+                                     true, y_dtype))
+    return st;
+  if (fp8_status_t st = check_device()) return st;
+  if (cudaMemsetAsync(y_amax, 0, sizeof(float), as_stream(stream)) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  if (T == 0) return FP8_OK;
+  return run_gemm(x8, fx, false, bias_x, w8, fw, false, bias_w, T, out, in, y, y_dtype,
+                  as_stream(stream), y_amax);
+}
+
+fp8_status_t fp8_linear_bwd_dgrad_amax(const uint8_t* dy8, fp8_format_t fdy,
+                                       const int32_t* bias_dy, const uint8_t* w8, fp8_format_t fw,
+                                       const int32_t* bias_w, int64_t T, int64_t in, int64_t out,
+                                       void* dx, fp8_dtype_t dx_dtype, float* dx_amax,
+                                       void* stream) {
+  if (!dx_amax) return FP8_ERR_INVALID_ARGUMENT;
+  if (reinterpret_cast<uintptr_t>(dx_amax) & 3u) return FP8_ERR_MISALIGNED;
+  if (fp8_status_t st = check_linear(dy8, true, fdy, bias_dy, w8, false, fw, bias_w, T, in, out,
+                                     dx, true, dx_dtype))
+    return st;
+  if (fp8_status_t st = check_device()) return st;
+  if (cudaMemsetAsync(dx_amax, 0, sizeof(float), as_stream(stream)) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  if (T == 0) return FP8_OK;
+  return run_gemm(dy8, fdy, false, bias_dy, w8, fw, true, bias_w, T, in, out, dx, dx_dtype,
+                  as_stream(stream), dx_amax);
 }
 
 fp8_status_t fp8_device_error(int clear, int32_t* where) {

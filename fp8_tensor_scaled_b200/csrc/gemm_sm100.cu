@@ -88,34 +88,41 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
-// Tile shapes.  kCta = 1: one CTA computes a 128 x 256 tile with
-// tcgen05.mma.cta_group::1 (M=128, N=256).  kCta = 2: a pair of CTAs (a
-// cluster of 2) computes a 256 x 256 tile with cta_group::2 (M=256, N=256):
-// CTA r loads rows [128r, 128r+128) of the A tile and of the B tile into its
-// own shared memory and holds rows [128r, 128r+128) of the accumulator in its
-// own tensor memory; the leader (r = 0) issues the MMAs for both.
-constexpr int BN = 256;                 // UMMA N
+// Tile shapes (kTile):
+//   kTileSingle  one CTA computes a 128 x 256 tile with tcgen05.mma.cta_group::1
+//                (M=128, N=256); B may be K- or MN-major.
+//   kTilePair    a pair of CTAs (a cluster of 2) computes a 256 x 256 tile with
+//                cta_group::2 (M=256, N=256): CTA r loads rows [128r, 128r+128)
+//                of the A tile and of the B tile into its own shared memory and
+//                holds rows [128r, 128r+128) of the accumulator in its own tensor
+//                memory; the leader (r = 0) issues the MMAs for both.
+//   kTileNarrow  one CTA computes a 128 x 64 tile (M=128, N=64), K-major B only:
+//                for few rows (decode-sized T) the GEMM streams the weights, and
+//                narrow tiles give every SM a share of them.
 constexpr int BK = 128;                 // K per stage: one 128-byte swizzle row of FP8
 constexpr int UK = 32;                  // K per tcgen05.mma of kind::f8f6f4
 constexpr uint32_t A_BYTES = 128 * BK;  // 16 KB: 128 rows of A per CTA
-constexpr uint32_t TMEM_COLS = 512;     // 2 accumulators x 256 fp32 columns
 constexpr int kThreads = 192;           // 6 warps
 
-template <int kCta> struct Cfg;
-template <> struct Cfg<1> {
-  static constexpr int BM = 128;                       // rows per tile
-  static constexpr uint32_t B_BYTES = BN * BK;         // 32 KB: all 256 B rows
-  static constexpr int STAGES = 4;
+enum TileKind : int { kTileSingle = 0, kTilePair = 1, kTileNarrow = 2 };
+
+template <int kTile> struct Cfg;
+template <> struct Cfg<kTileSingle> {
+  static constexpr int CTAS = 1, BM = 128, BN = 256, B_ROWS = 256, STAGES = 4;
 };
-template <> struct Cfg<2> {
-  static constexpr int BM = 256;
-  static constexpr uint32_t B_BYTES = (BN / 2) * BK;   // 16 KB: this CTA's 128 B rows
-  static constexpr int STAGES = 6;                     // 6 x 32 KB = 192 KB
+template <> struct Cfg<kTilePair> {
+  static constexpr int CTAS = 2, BM = 256, BN = 256, B_ROWS = 128, STAGES = 6;
 };
-template <int kCta> constexpr uint32_t stage_bytes() { return A_BYTES + Cfg<kCta>::B_BYTES; }
-template <int kCta> constexpr int num_bars() { return 2 * Cfg<kCta>::STAGES + 2 + 2 + 1; }
-template <int kCta> constexpr size_t smem_bytes() {
-  return 1024 + Cfg<kCta>::STAGES * stage_bytes<kCta>() + num_bars<kCta>() * 8 + 16;
+template <> struct Cfg<kTileNarrow> {
+  static constexpr int CTAS = 1, BM = 128, BN = 64, B_ROWS = 64, STAGES = 8;
+};
+template <int kTile> constexpr uint32_t b_bytes() { return Cfg<kTile>::B_ROWS * BK; }
+template <int kTile> constexpr uint32_t stage_bytes() { return A_BYTES + b_bytes<kTile>(); }
+// two fp32 accumulators of BN columns each
+template <int kTile> constexpr uint32_t tmem_cols() { return 2 * Cfg<kTile>::BN; }
+template <int kTile> constexpr int num_bars() { return 2 * Cfg<kTile>::STAGES + 2 + 2 + 1; }
+template <int kTile> constexpr size_t smem_bytes() {
+  return 1024 + Cfg<kTile>::STAGES * stage_bytes<kTile>() + num_bars<kTile>() * 8 + 16;
 }
 
 struct Params {
@@ -126,6 +133,7 @@ struct Params {
   const int32_t* bias_a;
   const int32_t* bias_b;
   void* d;
+  uint32_t* amax_out;        // fp32 bits of max |D|; used when the kernel has kAmax
   uint64_t wait_limit_ns;
 };
 
@@ -188,15 +196,23 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
-template <int kCta, bool kAMN, bool kBMN, bool kOutF32>
+// kAmax: the epilogue also takes the max of |D| over the values it stores
+// (after the rounding to the output type), reduces it per warp and combines
+// it into *p.amax_out with one atomicMax per warp (NaN > inf > finite, as in
+// the amax kernel), so the next layer's quantization needs no read of D.
+template <int kTile, bool kAMN, bool kBMN, bool kOutF32, bool kAmax>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b, const Params p) {
-  using C = Cfg<kCta>;
+  using C = Cfg<kTile>;
+  constexpr int kCta = C::CTAS;
+  constexpr int BN = C::BN;
   constexpr int STAGES = C::STAGES;
-  constexpr uint32_t B_BYTES = C::B_BYTES;
-  constexpr uint32_t STAGE_BYTES = stage_bytes<kCta>();
-  constexpr int kNumBars = num_bars<kCta>();
+  constexpr uint32_t B_BYTES = b_bytes<kTile>();
+  constexpr uint32_t STAGE_BYTES = stage_bytes<kTile>();
+  constexpr uint32_t TMEM_COLS = tmem_cols<kTile>();
+  constexpr int kNumBars = num_bars<kTile>();
+  static_assert(kTile != kTileNarrow || !kBMN, "narrow tiles take a K-major B only");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -357,6 +373,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
     const int row_in_tile = static_cast<int>(rank) * 128 + quarter * 32 + lane;
     const Pow2Scale sc = make_pow2_scale(-(*p.bias_a + *p.bias_b));
+    uint32_t dmax = 0;   // kAmax: this thread's max |D| bits (packed bf16 pair or fp32)
     int local = 0;
     for (int t = unit; t < p.num_tiles; t += num_units, ++local) {
       const int acc = local & 1;
@@ -392,6 +409,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 v.z = apply_pow2(__uint_as_float(r[4 * j + 2]), sc);
                 v.w = apply_pow2(__uint_as_float(r[4 * j + 3]), sc);
                 *reinterpret_cast<float4*>(dst + 4 * j) = v;
+                if (kAmax)
+                  dmax = max(dmax, max(max(__float_as_uint(v.x) & 0x7FFFFFFFu,
+                                           __float_as_uint(v.y) & 0x7FFFFFFFu),
+                                       max(__float_as_uint(v.z) & 0x7FFFFFFFu,
+                                           __float_as_uint(v.w) & 0x7FFFFFFFu)));
               }
             }
           } else {
@@ -409,6 +431,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 v.w = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 6]), sc),
                                   apply_pow2(__uint_as_float(r[8 * j + 7]), sc));
                 *reinterpret_cast<uint4*>(dst + 8 * j) = v;
+                if (kAmax) {
+                  dmax = __vmaxu2(dmax, v.x & 0x7FFF7FFFu);
+                  dmax = __vmaxu2(dmax, v.y & 0x7FFF7FFFu);
+                  dmax = __vmaxu2(dmax, v.z & 0x7FFF7FFFu);
+                  dmax = __vmaxu2(dmax, v.w & 0x7FFF7FFFu);
+                }
               }
             }
           }
@@ -420,6 +448,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (kCta == 2) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));  // leader's barrier
         else           mbar_arrive(tempty_bar(acc));
       }
+    }
+    if (kAmax) {
+      // a bf16 is the top half of an fp32: widen the packed pair's max
+      uint32_t bits = kOutF32 ? dmax : (max(dmax & 0xFFFFu, dmax >> 16) << 16);
+      bits = __reduce_max_sync(0xFFFFFFFFu, bits);
+      if (lane == 0 && bits != 0u) atomicMax(p.amax_out, bits);
     }
   }
 
@@ -508,13 +542,16 @@ int sm_count() {
 // evict-last hint on either operand only slowed it down.
 constexpr int kGroupN = 16;
 
-template <int kCta, bool kAMN, bool kBMN, bool kOutF32>
+template <int kTile, bool kAMN, bool kBMN, bool kOutF32, bool kAmax>
 int launch_t(const GemmArgs& g, cudaStream_t s) {
-  constexpr int BM = Cfg<kCta>::BM;
-  constexpr size_t kSmem = smem_bytes<kCta>();
-  // TMA boxes: 128 x 128 bytes for A (this CTA's rows) and, for B, all 256
-  // rows (one CTA, K-major) or 128 rows / MN columns (MN-major, or a pair).
-  const uint32_t b_box_rows = (kCta == 1 && !kBMN) ? BN : 128;
+  constexpr int kCta = Cfg<kTile>::CTAS;
+  constexpr int BM = Cfg<kTile>::BM;
+  constexpr int BN = Cfg<kTile>::BN;
+  constexpr size_t kSmem = smem_bytes<kTile>();
+  // TMA boxes: 128 x 128 bytes for A (this CTA's rows); for a K-major B, the
+  // CTA's B rows (256, 128 or 64) x 128 bytes; for an MN-major B, 128 MN
+  // columns x 128 K rows (the single-CTA tile loads two of them).
+  const uint32_t b_box_rows = kBMN ? 128 : Cfg<kTile>::B_ROWS;
   CUtensorMap ta, tb;
   const uint64_t M = g.M, N = g.N, K = g.K;
   const bool ok_a = kAMN ? encode_2d(&ta, g.a, M, K, 128, BK) : encode_2d(&ta, g.a, K, M, BK, 128);
@@ -541,13 +578,14 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
   p.bias_a = g.bias_a;
   p.bias_b = g.bias_b;
   p.d = g.d;
+  p.amax_out = reinterpret_cast<uint32_t*>(g.d_amax);
   p.wait_limit_ns = kWaitLimitNs;
 
   static int max_units[64];      // co-resident CTAs (1-CTA) or clusters (pair), per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  auto kern = fp8_gemm_kernel<kCta, kAMN, kBMN, kOutF32>;
+  auto kern = fp8_gemm_kernel<kTile, kAMN, kBMN, kOutF32, kAmax>;
 
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -584,20 +622,40 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
   return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
-template <bool kAMN, bool kBMN, bool kOutF32>
+template <bool kAMN, bool kBMN, bool kOutF32, bool kAmax = false>
 int launch_pick(const GemmArgs& g, cudaStream_t s) {
-  // One 128-row tile covers M: a single CTA per tile; otherwise CTA pairs.
-  if (g.M <= 128) return launch_t<1, kAMN, kBMN, kOutF32>(g, s);
-  return launch_t<2, kAMN, kBMN, kOutF32>(g, s);
+  // One 128-row tile covers M: single-CTA tiles; otherwise CTA pairs.  With
+  // so few rows the GEMM streams B, and every SM should get a share of it:
+  // narrow 128 x 64 tiles are used when 128 x 256 tiles would leave more than
+  // half of the SMs idle and the narrow ones still fit in one wave (measured on
+  // the Llama-2-70B projections at T <= 128: a second, mostly empty wave of
+  // narrow tiles costs more than the idle SMs of the wide ones).
+  if (g.M <= 128) {
+    const int64_t wide = (g.N + 255) / 256, narrow = (g.N + 63) / 64;
+    if (!kBMN && 2 * wide < sm_count() && narrow <= sm_count())
+      return launch_t<kTileNarrow, kAMN, false, kOutF32, kAmax>(g, s);
+    return launch_t<kTileSingle, kAMN, kBMN, kOutF32, kAmax>(g, s);
+  }
+  return launch_t<kTilePair, kAMN, kBMN, kOutF32, kAmax>(g, s);
 }
 
 }  // namespace
 
 int launch_gemm(const GemmArgs& g, cudaStream_t s) {
   // limits of the 32-bit tile arithmetic and of the TMA tensor map
-  if (g.M > (1LL << 31) - 1 - 256 || g.N > (1LL << 31) - 1 - BN || g.K > (1LL << 31) - 1 - BK)
+  if (g.M > (1LL << 31) - 1 - 256 || g.N > (1LL << 31) - 1 - 256 || g.K > (1LL << 31) - 1 - BK)
     return FP8_ERR_UNSUPPORTED;
   const int key = (g.a_mn_major ? 4 : 0) | (g.b_mn_major ? 2 : 0) | (g.d_fp32 ? 1 : 0);
+  if (g.d_amax) {
+    // output amax: the passes whose output feeds another quantization (fwd, dgrad)
+    switch (key) {
+      case 0: return launch_pick<false, false, false, true>(g, s);
+      case 1: return launch_pick<false, false, true, true>(g, s);
+      case 2: return launch_pick<false, true, false, true>(g, s);
+      case 3: return launch_pick<false, true, true, true>(g, s);
+      default: return FP8_ERR_UNSUPPORTED;
+    }
+  }
   switch (key) {
     case 0: return launch_pick<false, false, false>(g, s);
     case 1: return launch_pick<false, false, true>(g, s);

@@ -27,6 +27,7 @@ struct GemmArgs {
   const int32_t* bias_b;
   void* d;
   bool d_fp32;
+  float* d_amax;   // optional: receives max |D| (must be zeroed before the launch)
   int64_t M, N, K;
 };
 

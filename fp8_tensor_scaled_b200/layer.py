@@ -7,7 +7,13 @@ are cast to FP8_E4 (E4M3), gradients to FP8_E5 (E5M2); the matmuls run on the
 FP8 operands and their outputs are unscaled by 2^-(biasA + biasB).
 
 ``Fp8AmaxLinear`` owns the FP8 buffers and the per-tensor scalars of one
-linear [in -> out] at T tokens, so that a step allocates nothing:
+linear [in -> out] at T tokens, so that a step allocates nothing.  Two options
+follow the page's comparison of scaling policies ("Proposed method" and the
+research questions on how often the bias must be updated):
+  * ``bias_update_every=k``: amax and bias are recomputed on every k-th
+    step only; the steps in between cast with the stored biases and skip the
+    amax pass (k = 1 is FP8-AMAX proper);
+  * ``fixed_bias=(bx, bw, bdy)``: FP8-CSCALE, constant biases, no amax at all.
 
     step(x, w, dy)  ->  quantize X (E4M3), W (E4M3), dY (E5M2)
                         Y  = X8 . W8^T        (fwd)
@@ -18,16 +24,22 @@ Every operation is one call of the C library (see ``__init__``).
 """
 import torch
 
-from . import (E4M3, E5M2, fp8_linear_bwd_dgrad, fp8_linear_bwd_wgrad, fp8_linear_fwd,
-               fp8_quantize)
+from . import (E4M3, E5M2, fp8_cast_scaled, fp8_linear_bwd_dgrad, fp8_linear_bwd_wgrad,
+               fp8_linear_fwd, fp8_quantize)
 
 
 class Fp8AmaxLinear:
     def __init__(self, tokens, in_features, out_features, device, out_dtype=torch.bfloat16,
-                 margin_x=0, margin_w=0, margin_dy=0, backward=True):
+                 margin_x=0, margin_w=0, margin_dy=0, backward=True, bias_update_every=1,
+                 fixed_bias=None):
         self.T, self.inf, self.outf = int(tokens), int(in_features), int(out_features)
         self.margins = (int(margin_x), int(margin_w), int(margin_dy))
         self.backward = backward
+        if int(bias_update_every) < 1:
+            raise ValueError("bias_update_every must be >= 1")
+        self.every = int(bias_update_every)
+        self.fixed = tuple(int(b) for b in fixed_bias) if fixed_bias is not None else None
+        self.calls = 0
         dev = torch.device(device)
         u8 = dict(dtype=torch.uint8, device=dev)
         self.x8 = torch.empty((self.T, self.inf), **u8)
@@ -35,6 +47,10 @@ class Fp8AmaxLinear:
         # one buffer for the 3 amax values and one for the 3 biases (X, W, dY)
         self.amax = torch.zeros(3, dtype=torch.float32, device=dev)
         self.bias = torch.zeros(3, dtype=torch.int32, device=dev)
+        if self.fixed is not None:
+            if len(self.fixed) != 3:
+                raise ValueError("fixed_bias is (bias_x, bias_w, bias_dy)")
+            self.bias.copy_(torch.tensor(self.fixed, dtype=torch.int32))
         self.y = torch.empty((self.T, self.outf), dtype=out_dtype, device=dev)
         if backward:
             self.dy8 = torch.empty((self.T, self.outf), **u8)
@@ -42,11 +58,18 @@ class Fp8AmaxLinear:
             self.dw = torch.empty((self.outf, self.inf), dtype=out_dtype, device=dev)
 
     def quantize(self, x, w, dy=None):
-        mx, mw, mdy = self.margins
-        fp8_quantize(x, E4M3, mx, self.amax[0:1], self.bias[0:1], self.x8)
-        fp8_quantize(w, E4M3, mw, self.amax[1:2], self.bias[1:2], self.w8)
+        """Cast X, W (E4M3) and dY (E5M2).  On refresh steps amax -> bias ->
+        cast (fp8_quantize); otherwise cast with the stored bias."""
+        refresh = self.fixed is None and self.calls % self.every == 0
+        self.calls += 1
+        work = [(x, E4M3, 0, self.x8), (w, E4M3, 1, self.w8)]
         if self.backward:
-            fp8_quantize(dy, E5M2, mdy, self.amax[2:3], self.bias[2:3], self.dy8)
+            work.append((dy, E5M2, 2, self.dy8))
+        for t, fmt, i, out in work:
+            if refresh:
+                fp8_quantize(t, fmt, self.margins[i], self.amax[i:i + 1], self.bias[i:i + 1], out)
+            else:
+                fp8_cast_scaled(t, self.bias[i:i + 1], fmt, out=out)
 
     def gemms(self):
         bx, bw, bdy = self.bias[0:1], self.bias[1:2], self.bias[2:3]

@@ -129,6 +129,27 @@ fp8_status_t fp8_linear_bwd_wgrad(const uint8_t *dy8, fp8_format_t fdy, const in
                                   int64_t T, int64_t in, int64_t out,
                                   void *dw, fp8_dtype_t dw_dtype, void *stream);
 
+/*
+ * fwd and dgrad with the amax of their output fused into the GEMM epilogue
+ * (the output of one linear is the input of the next, whose FP8-AMAX cast
+ * needs that amax).  Same results in y / dx as fp8_linear_fwd /
+ * fp8_linear_bwd_dgrad; in addition *y_amax / *dx_amax (one float, device,
+ * 4-byte aligned) receives max |value| over the output exactly as stored
+ * (after its rounding to BF16/FP32), with fp8_amax's NaN/inf rules, so it is
+ * bit-identical to calling fp8_amax on the output, without reading it back.
+ * T == 0 writes 0.
+ */
+fp8_status_t fp8_linear_fwd_amax(const uint8_t *x8, fp8_format_t fx, const int32_t *bias_x,
+                                 const uint8_t *w8, fp8_format_t fw, const int32_t *bias_w,
+                                 int64_t T, int64_t in, int64_t out,
+                                 void *y, fp8_dtype_t y_dtype, float *y_amax, void *stream);
+
+fp8_status_t fp8_linear_bwd_dgrad_amax(const uint8_t *dy8, fp8_format_t fdy,
+                                       const int32_t *bias_dy, const uint8_t *w8, fp8_format_t fw,
+                                       const int32_t *bias_w, int64_t T, int64_t in, int64_t out,
+                                       void *dx, fp8_dtype_t dx_dtype, float *dx_amax,
+                                       void *stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *fp8_status_string(fp8_status_t status);
 

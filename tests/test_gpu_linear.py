@@ -213,3 +213,82 @@ def test_bounded_wait_selftest_and_error_word():
     # the context is still usable afterwards
     x = torch.ones(1024, device=DEV)
     assert fp8.fp8_amax(x).item() == 1.0
+
+
+@pytest.mark.parametrize("T,In,Out", [(200, 272, 400), (128, 256, 256), (333, 256, 528), (1, 16, 16)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_fused_output_amax(T, In, Out, out_dtype):
+    """fwd / dgrad with the output amax taken in the epilogue: the output is
+    bit-identical to the plain call and the amax is exactly max |stored value|
+    (checked against the oracle's amax of the GPU output and fp8_amax)."""
+    x, w, dy = _inputs(T, In, Out, seed=11 + T)
+    Q = _passes(x, w, dy)
+    qx, bx, _, _, fx = Q["x"]
+    qw, bw, _, _, fw = Q["w"]
+    qdy, bdy, _, _, fdy = Q["dy"]
+    y, ya = fp8.fp8_linear_fwd(qx, fx, bx, qw, fw, bw, out_dtype=out_dtype, amax=True)
+    y0 = fp8.fp8_linear_fwd(qx, fx, bx, qw, fw, bw, out_dtype=out_dtype)
+    dx, dxa = fp8.fp8_linear_bwd_dgrad(qdy, fdy, bdy, qw, fw, bw, out_dtype=out_dtype, amax=True)
+    dx0 = fp8.fp8_linear_bwd_dgrad(qdy, fdy, bdy, qw, fw, bw, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    for got, plain, a in ((y, y0, ya), (dx, dx0, dxa)):
+        assert torch.equal(got.view(torch.int16 if out_dtype == torch.bfloat16 else torch.int32),
+                           plain.view(torch.int16 if out_dtype == torch.bfloat16 else torch.int32))
+        ref = oracle.amax(got.cpu())
+        assert np.float32(a.item()) == ref
+        assert fp8.fp8_amax(got).item() == a.item()
+    # both passes also against the oracle's GEMM
+    _compare_full(oracle.FWD, Q, T, In, Out, out_dtype, "fwd+amax")
+
+
+def test_fused_output_amax_empty_and_c3():
+    b = torch.zeros(1, dtype=torch.int32, device=DEV)
+    z8 = torch.empty((0, 64), dtype=torch.uint8, device=DEV)
+    w8 = torch.zeros((32, 64), dtype=torch.uint8, device=DEV)
+    a = torch.full((1,), 5.0, device=DEV)
+    y, ya = fp8.fp8_linear_fwd(z8, E4, b, w8, E4, b, amax=a)
+    torch.cuda.synchronize()
+    assert ya.item() == 0.0
+    # the Llama-2-70B gate projection, fwd and dgrad
+    cfg = workloads.C3
+    x, w, dy = workloads.linear_inputs(3, 1)
+    Q = _passes(x, w, dy)
+    qx, bx, _, _, fx = Q["x"]
+    qw, bw, _, _, fw = Q["w"]
+    qdy, bdy, _, _, fdy = Q["dy"]
+    y, ya = fp8.fp8_linear_fwd(qx, fx, bx, qw, fw, bw, amax=True)
+    dx, dxa = fp8.fp8_linear_bwd_dgrad(qdy, fdy, bdy, qw, fw, bw, amax=True)
+    torch.cuda.synchronize()
+    assert fp8.fp8_amax(y).item() == ya.item()
+    assert fp8.fp8_amax(dx).item() == dxa.item()
+    assert np.float32(ya.item()) == oracle.amax(y.cpu())
+
+
+def test_bias_update_every_k_and_fixed_bias():
+    """Bias recomputed every k-th step only (the page's update-frequency
+    question), and FP8-CSCALE fixed biases: the codes the layer casts are the
+    oracle's cast with the bias that should be in force at that step."""
+    T, In, Out = 96, 128, 160
+    layer = fp8.Fp8AmaxLinear(T, In, Out, DEV, bias_update_every=3)
+    fixed = fp8.Fp8AmaxLinear(T, In, Out, DEV, fixed_bias=(2, 9, 20))
+    held = None
+    for step in range(5):
+        scale = 4.0 ** step                    # amax changes every step
+        x, w, dy = _inputs(T, In, Out, seed=300 + step, x_scale=scale)
+        layer.step(x.to(DEV), w.to(DEV), dy.to(DEV))
+        fixed.step(x.to(DEV), w.to(DEV), dy.to(DEV))
+        torch.cuda.synchronize()
+        if step % 3 == 0:
+            held = [oracle.quantize(t, f, 0)[1] for t, f in ((x, E4), (w, E4), (dy, E5))]
+        assert layer.bias.cpu().tolist() == held, step
+        for t, f, i, buf in ((x, E4, 0, layer.x8), (w, E4, 1, layer.w8), (dy, E5, 2, layer.dy8)):
+            ref = oracle.cast_scaled(t, held[i], f).reshape(tuple(t.shape))
+            assert codes_equal_nan_aware(u8(buf), ref, f), (step, i)
+        for t, f, i, buf in ((x, E4, 0, fixed.x8), (w, E4, 1, fixed.w8), (dy, E5, 2, fixed.dy8)):
+            ref = oracle.cast_scaled(t, (2, 9, 20)[i], f).reshape(tuple(t.shape))
+            assert codes_equal_nan_aware(u8(buf), ref, f), (step, i)
+        assert fixed.bias.cpu().tolist() == [2, 9, 20]
+        # and the GEMM on those codes is the oracle's
+        ref, absref = oracle.linear(oracle.FWD, u8(layer.x8), E4, held[0], u8(layer.w8), E4,
+                                    held[1], T, In, Out)
+        assert_gemm_close(to_f64(layer.y), ref, absref, "every-3 fwd step %d" % step)
