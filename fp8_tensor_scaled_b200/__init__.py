@@ -62,6 +62,8 @@ def lib():
                                 vp],
         "fp8_linear_bwd_dgrad_amax": [vp, c.c_int, vp, vp, c.c_int, vp, i64, i64, i64, vp, c.c_int,
                                       vp, vp],
+        "fp8_linear_fwd_ws": [vp, c.c_int, vp, vp, c.c_int, vp, i64, i64, i64, vp, c.c_int, vp,
+                              sz, vp],
         "fp8_device_error": [c.c_int, vp],
         "fp8_selftest_bounded_wait": [u64],
         "fp8_abi_version": [],
@@ -72,6 +74,8 @@ def lib():
         f.restype = c.c_int
     L.fp8_status_string.argtypes = [c.c_int]
     L.fp8_status_string.restype = c.c_char_p
+    L.fp8_linear_fwd_workspace_size.argtypes = [i64, i64, i64]
+    L.fp8_linear_fwd_workspace_size.restype = sz
     _lib = L
     return L
 
@@ -202,6 +206,33 @@ def fp8_linear_fwd(x8, fx, bias_x, w8, fw, bias_w, out=None, out_dtype=torch.bfl
                    out, out_dtype, amax)
 
 
+def fp8_linear_fwd_workspace_size(T, in_, out_):
+    """Bytes of workspace fp8_linear_fwd_ws splits K with (0: no split)."""
+    return int(lib().fp8_linear_fwd_workspace_size(int(T), int(in_), int(out_)))
+
+
+def fp8_linear_fwd_ws(x8, fx, bias_x, w8, fw, bias_w, out=None, out_dtype=torch.bfloat16,
+                      workspace=None):
+    """fp8_linear_fwd for few tokens with a split-K workspace (allocated here
+    through torch when not given)."""
+    T, in_ = x8.shape
+    out_ = w8.shape[0]
+    assert w8.shape[1] == in_
+    _need_cuda(x8, bias_x, w8, bias_w, out, workspace)
+    dev = bias_x.device
+    if out is None:
+        out = torch.empty((T, out_), dtype=out_dtype, device=dev)
+    need = fp8_linear_fwd_workspace_size(T, in_, out_)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("fp8_linear_fwd_ws", lib().fp8_linear_fwd_ws(
+        _ptr(x8), int(fx), _ptr(bias_x), _ptr(w8), int(fw), _ptr(bias_w), int(T), int(in_),
+        int(out_), _ptr(out), _OUT[out.dtype], _ptr(workspace), nbytes,
+        ctypes.c_void_p(_stream_ptr(bias_x))))
+    return out
+
+
 def fp8_linear_bwd_dgrad(dy8, fdy, bias_dy, w8, fw, bias_w, out=None, out_dtype=torch.bfloat16,
                          amax=False):
     """dX [T,in] = (dY8 [T,out] . W8 [out,in]) * 2^-(bias_dy + bias_w).
@@ -242,5 +273,6 @@ __all__ = [
     "E4M3", "E5M2", "BF16", "FP32", "FMT_MAX", "Fp8Error", "lib", "declared_entry_points",
     "fp8_status_string", "fp8_amax", "fp8_compute_bias", "fp8_cast_scaled", "fp8_quantize",
     "fp8_linear_fwd", "fp8_linear_bwd_dgrad", "fp8_linear_bwd_wgrad", "fp8_device_error",
+    "fp8_linear_fwd_ws", "fp8_linear_fwd_workspace_size",
     "fp8_selftest_bounded_wait", "Fp8AmaxLinear",
 ]

@@ -129,6 +129,15 @@ struct Params {
   int M, N, K;
   int num_m_blocks, num_n_blocks, num_k_blocks, num_tiles;
   int group_n;
+  // Split K: each tile's K range is cut into `splits` ranges of kb_per_split
+  // k-blocks; work unit u is (tile u / splits, range u % splits).  With
+  // splits > 1 every unit writes its fp32 partial to ws[range][M][N], and for
+  // each 32-row quarter of a tile the last unit to finish it (counted in
+  // counters[tile * 4 + quarter]) adds the partials in range order and runs
+  // the epilogue on those rows.
+  int splits, kb_per_split, num_work;
+  float* ws;
+  uint32_t* counters;
   uint32_t idesc;
   const int32_t* bias_a;
   const int32_t* bias_b;
@@ -192,6 +201,57 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
       *abort_flag = 1;
       record_device_error(site);
       return false;
+    }
+  }
+}
+
+// Scale, round and store one row's 32 consecutive accumulator columns
+// (fp32 bits in r) at D[row, col0 ..]; with kAmax also fold max |stored| into
+// dmax (fp32 bits, or two packed bf16 maxima).
+template <bool kOutF32, bool kAmax>
+__device__ __forceinline__ void store_row_chunk(const Params& p, int64_t row, int col0,
+                                                const uint32_t (&r)[32], const Pow2Scale& sc,
+                                                uint32_t& dmax) {
+  if (kOutF32) {
+    float* dst = static_cast<float*>(p.d) + row * p.N + col0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (col0 + 4 * j < p.N) {
+        float4 v;
+        v.x = apply_pow2(__uint_as_float(r[4 * j + 0]), sc);
+        v.y = apply_pow2(__uint_as_float(r[4 * j + 1]), sc);
+        v.z = apply_pow2(__uint_as_float(r[4 * j + 2]), sc);
+        v.w = apply_pow2(__uint_as_float(r[4 * j + 3]), sc);
+        *reinterpret_cast<float4*>(dst + 4 * j) = v;
+        if (kAmax)
+          dmax = max(dmax, max(max(__float_as_uint(v.x) & 0x7FFFFFFFu,
+                                   __float_as_uint(v.y) & 0x7FFFFFFFu),
+                               max(__float_as_uint(v.z) & 0x7FFFFFFFu,
+                                   __float_as_uint(v.w) & 0x7FFFFFFFu)));
+      }
+    }
+  } else {
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.d) + row * p.N + col0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (col0 + 8 * j < p.N) {
+        uint4 v;
+        v.x = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 0]), sc),
+                          apply_pow2(__uint_as_float(r[8 * j + 1]), sc));
+        v.y = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 2]), sc),
+                          apply_pow2(__uint_as_float(r[8 * j + 3]), sc));
+        v.z = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 4]), sc),
+                          apply_pow2(__uint_as_float(r[8 * j + 5]), sc));
+        v.w = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 6]), sc),
+                          apply_pow2(__uint_as_float(r[8 * j + 7]), sc));
+        *reinterpret_cast<uint4*>(dst + 8 * j) = v;
+        if (kAmax) {
+          dmax = __vmaxu2(dmax, v.x & 0x7FFF7FFFu);
+          dmax = __vmaxu2(dmax, v.y & 0x7FFF7FFFu);
+          dmax = __vmaxu2(dmax, v.z & 0x7FFF7FFFu);
+          dmax = __vmaxu2(dmax, v.w & 0x7FFF7FFFu);
+        }
+      }
     }
   }
 }
@@ -274,13 +334,16 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     int stage = 0;
     uint32_t phase = 0;
     uint32_t armed_mask = 0, armed_parity = 0;   // leader: last armed phase per stage
-    for (int t = unit; t < p.num_tiles && !*abort_flag; t += num_units) {
+    for (int u = unit; u < p.num_work && !*abort_flag; u += num_units) {
+      const int t = u / p.splits;
+      const int kb0 = (u - t * p.splits) * p.kb_per_split;
+      const int kb1 = min(kb0 + p.kb_per_split, p.num_k_blocks);
       int mb, nb;
       tile_coords(t, p, mb, nb);
       const int a_row = mb * C::BM + static_cast<int>(rank) * 128;
       const int b_row = nb * BN + (kCta == 2 ? static_cast<int>(rank) * 128 : 0);
       bool ok = true;
-      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!wait_bar<kCta>(empty_bar(stage), phase ^ 1u, abort_flag, kSiteProducerEmpty,
                             p.wait_limit_ns)) {
           ok = false;
@@ -329,7 +392,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     int stage = 0;
     uint32_t phase = 0;
     int local = 0;
-    for (int t = unit; t < p.num_tiles; t += num_units, ++local) {
+    for (int u = unit; u < p.num_work; u += num_units, ++local) {
+      const int t = u / p.splits;
+      const int kb0 = (u - t * p.splits) * p.kb_per_split;
+      const int kb1 = min(kb0 + p.kb_per_split, p.num_k_blocks);
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       if (!wait_bar<kCta>(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, kSiteMmaTmemEmpty,
@@ -338,7 +404,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
       bool ok = true;
-      for (int kb = 0; kb < p.num_k_blocks; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!wait_bar<kCta>(full_bar(stage), phase, abort_flag, kSiteMmaFull, p.wait_limit_ns)) {
           ok = false;
           break;
@@ -350,8 +416,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         for (int k = 0; k < BK / UK; ++k) {
           const uint64_t ad = operand_desc<kAMN>(a_base, k);
           const uint64_t bd = operand_desc<kBMN>(b_base, k);
-          if (kCta == 2) mma_f8f6f4_pair(d_tmem, ad, bd, p.idesc, (kb | k) != 0 ? 1u : 0u);
-          else           mma_f8f6f4(d_tmem, ad, bd, p.idesc, (kb | k) != 0 ? 1u : 0u);
+          const uint32_t accum = (kb != kb0 || k != 0) ? 1u : 0u;
+          if (kCta == 2) mma_f8f6f4_pair(d_tmem, ad, bd, p.idesc, accum);
+          else           mma_f8f6f4(d_tmem, ad, bd, p.idesc, accum);
         }
         // frees the stage (in both CTAs) once these MMAs have read it
         if (kCta == 2) mma_commit_pair_mc(empty_bar(stage), 0x3);
@@ -375,7 +442,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     const Pow2Scale sc = make_pow2_scale(-(*p.bias_a + *p.bias_b));
     uint32_t dmax = 0;   // kAmax: this thread's max |D| bits (packed bf16 pair or fp32)
     int local = 0;
-    for (int t = unit; t < p.num_tiles; t += num_units, ++local) {
+    for (int u = unit; u < p.num_work; u += num_units, ++local) {
+      const int t = u / p.splits;
+      const int split = u - t * p.splits;
       const int acc = local & 1;
       const uint32_t use = static_cast<uint32_t>(local >> 1);
       int ok = 1;
@@ -389,6 +458,65 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       tile_coords(t, p, mb, nb);
       const int64_t row = static_cast<int64_t>(mb) * C::BM + row_in_tile;
       const bool row_ok = row < p.M;
+      if (kCta == 1 && p.splits > 1) {
+        // ---- split K: store this range's raw fp32 partial, free the
+        // accumulator, and let the last range to finish these 32 rows of the
+        // tile (one counter per tile and warp quarter, so the four epilogue
+        // warps never wait on each other) add the partials and store them
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col0 = nb * BN + c * 32;
+          if (col0 >= p.N) break;
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                 static_cast<uint32_t>(acc * BN + c * 32), r);
+          tmem_ld_wait();
+          if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(
+                p.ws + (static_cast<int64_t>(split) * p.M + row) * p.N + col0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              if (col0 + 4 * j < p.N)
+                __stcg(dst + j, make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                            __uint_as_float(r[4 * j + 2]),
+                                            __uint_as_float(r[4 * j + 3])));
+          }
+        }
+        tc_fence_before();
+        __threadfence();                          // partial visible before the count
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(acc));
+        uint32_t prev = 0;
+        if (lane == 0) prev = atomicAdd(&p.counters[t * 4 + quarter], 1u);
+        prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
+        if (prev != static_cast<uint32_t>(p.splits - 1)) continue;
+        __threadfence();                          // all partials visible to this warp
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col0 = nb * BN + c * 32;
+          if (col0 >= p.N) break;
+          if (!row_ok) continue;
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0.0f;
+          for (int sp = 0; sp < p.splits; ++sp) {     // fixed order: deterministic sum
+            const float4* src = reinterpret_cast<const float4*>(
+                p.ws + (static_cast<int64_t>(sp) * p.M + row) * p.N + col0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              if (col0 + 4 * j < p.N) {
+                const float4 q = __ldcg(src + j);
+                v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
+              }
+            }
+          }
+          uint32_t r[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(v[j]);
+          store_row_chunk<kOutF32, kAmax>(p, row, col0, r, sc, dmax);
+        }
+        continue;
+      }
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         const int col0 = nb * BN + c * 32;
@@ -397,50 +525,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                static_cast<uint32_t>(acc * BN + c * 32), r);
         tmem_ld_wait();
-        if (row_ok) {
-          if (kOutF32) {
-            float* dst = static_cast<float*>(p.d) + row * p.N + col0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (col0 + 4 * j < p.N) {
-                float4 v;
-                v.x = apply_pow2(__uint_as_float(r[4 * j + 0]), sc);
-                v.y = apply_pow2(__uint_as_float(r[4 * j + 1]), sc);
-                v.z = apply_pow2(__uint_as_float(r[4 * j + 2]), sc);
-                v.w = apply_pow2(__uint_as_float(r[4 * j + 3]), sc);
-                *reinterpret_cast<float4*>(dst + 4 * j) = v;
-                if (kAmax)
-                  dmax = max(dmax, max(max(__float_as_uint(v.x) & 0x7FFFFFFFu,
-                                           __float_as_uint(v.y) & 0x7FFFFFFFu),
-                                       max(__float_as_uint(v.z) & 0x7FFFFFFFu,
-                                           __float_as_uint(v.w) & 0x7FFFFFFFu)));
-              }
-            }
-          } else {
-            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.d) + row * p.N + col0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              if (col0 + 8 * j < p.N) {
-                uint4 v;
-                v.x = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 0]), sc),
-                                  apply_pow2(__uint_as_float(r[8 * j + 1]), sc));
-                v.y = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 2]), sc),
-                                  apply_pow2(__uint_as_float(r[8 * j + 3]), sc));
-                v.z = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 4]), sc),
-                                  apply_pow2(__uint_as_float(r[8 * j + 5]), sc));
-                v.w = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 6]), sc),
-                                  apply_pow2(__uint_as_float(r[8 * j + 7]), sc));
-                *reinterpret_cast<uint4*>(dst + 8 * j) = v;
-                if (kAmax) {
-                  dmax = __vmaxu2(dmax, v.x & 0x7FFF7FFFu);
-                  dmax = __vmaxu2(dmax, v.y & 0x7FFF7FFFu);
-                  dmax = __vmaxu2(dmax, v.z & 0x7FFF7FFFu);
-                  dmax = __vmaxu2(dmax, v.w & 0x7FFF7FFFu);
-                }
-              }
-            }
-          }
-        }
+        if (row_ok) store_row_chunk<kOutF32, kAmax>(p, row, col0, r, sc, dmax);
       }
       tc_fence_before();
       __syncwarp();
@@ -536,11 +621,44 @@ int sm_count() {
 // Tile order.  Tiles are walked in groups of `group_n` N-blocks, N fastest
 // inside a group; the clusters running at one time cover a window of about
 // 74 consecutive tiles, i.e. group_n N-blocks x 74/group_n M-blocks, whose
-// panels they share in L2.  Measured on the Llama-2-70B projections (all 12
-// GEMMs of a step, same clocks): group_n = 16 beat 8, 4, and the orders that
-// sweep one whole operand (M fastest or N fastest) by 1-5 %, and an
-// evict-last hint on either operand only slowed it down.
-constexpr int kGroupN = 16;
+// panels they share in L2.  Measured on the Llama-2-70B projections (each of
+// the 12 GEMMs of a step, same clocks): group_n = 16 beat 8, 4 and the orders
+// that sweep one whole operand (M fastest or N fastest) by 1-5 %, except
+// where both operands are large (K = 28672: both > 128 MB), where 8 won by
+// 1-2 %; an evict-last hint on either operand only slowed it down.
+// Split-K workspace: fp32 partials [splits][M][N] (256-byte aligned), then
+// one uint32 counter per tile and epilogue warp (4 per tile).
+size_t splitk_partials_bytes(int splits, int64_t M, int64_t N) {
+  return ((static_cast<size_t>(splits) * M * N * sizeof(float)) + 255) & ~size_t(255);
+}
+size_t splitk_workspace_bytes(int splits, int64_t M, int64_t N, int num_tiles) {
+  return splitk_partials_bytes(splits, M, N) + 4 * sizeof(uint32_t) * static_cast<size_t>(num_tiles);
+}
+
+int pick_group_n(uint64_t a_bytes, uint64_t b_bytes) {
+  return (a_bytes > (128ull << 20) && b_bytes > (128ull << 20)) ? 8 : 16;
+}
+
+// Split K for problems whose tiles cannot fill the GPU (few rows: the
+// weight-streaming GEMMs of decode).  Cut K into ranges so that tiles x splits
+// work units still fit in one wave.  Measured on the Llama-2-70B projections
+// (T = 1 .. 128): splitting pays only for long K ranges and few rows (down,
+// K = 28672, T <= 64: 2.3-3.2 -> 3.6-4.3 TB/s of weights), while short ranges
+// (QKV, K = 8192) and T = 128 lost to the fp32 partial traffic; hence at most
+// 64 rows and at least 48 k-blocks per range.  Returns 1 for no split.
+int plan_splits(int64_t M, int num_tiles, int num_k_blocks, int* kb_per_split) {
+  const int sms = sm_count();
+  int splits = 1;
+  if (M <= 64 && 2 * num_tiles <= sms) {
+    splits = sms / num_tiles;
+    splits = splits < num_k_blocks / 48 ? splits : num_k_blocks / 48;
+    splits = splits < 16 ? splits : 16;
+    if (splits < 1) splits = 1;
+  }
+  int per = (num_k_blocks + splits - 1) / splits;
+  *kb_per_split = per;
+  return (num_k_blocks + per - 1) / per;     // no empty range
+}
 
 template <int kTile, bool kAMN, bool kBMN, bool kOutF32, bool kAmax>
 int launch_t(const GemmArgs& g, cudaStream_t s) {
@@ -567,7 +685,27 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
   p.num_n_blocks = (p.N + BN - 1) / BN;
   p.num_k_blocks = (p.K + BK - 1) / BK;
   p.num_tiles = p.num_m_blocks * p.num_n_blocks;
-  p.group_n = kGroupN;
+  p.group_n = pick_group_n(M * K, N * K);
+  p.splits = 1;
+  p.kb_per_split = p.num_k_blocks;
+  p.ws = nullptr;
+  p.counters = nullptr;
+  if (g.workspace != nullptr && kCta == 1) {
+    int per = 0;
+    const int sp = plan_splits(g.M, p.num_tiles, p.num_k_blocks, &per);
+    if (sp > 1) {
+      const size_t need = splitk_workspace_bytes(sp, g.M, g.N, p.num_tiles);
+      if (need > g.workspace_bytes) return FP8_ERR_INVALID_ARGUMENT;
+      p.splits = sp;
+      p.kb_per_split = per;
+      p.ws = static_cast<float*>(g.workspace);
+      p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(g.workspace) +
+                                               splitk_partials_bytes(sp, g.M, g.N));
+      if (cudaMemsetAsync(p.counters, 0, 4 * sizeof(uint32_t) * p.num_tiles, s) != cudaSuccess)
+        return FP8_ERR_CUDA;
+    }
+  }
+  p.num_work = p.num_tiles * p.splits;
   p.idesc = (1u << 4)                                      // D = fp32
             | (static_cast<uint32_t>(g.a_fmt) << 7)       // A: 0 E4M3, 1 E5M2
             | (static_cast<uint32_t>(g.b_fmt) << 10)      // B: 0 E4M3, 1 E5M2
@@ -616,23 +754,28 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
     }
     max_units[dev] = units;
   }
-  const int units = p.num_tiles < max_units[dev] ? p.num_tiles : max_units[dev];
+  const int units = p.num_work < max_units[dev] ? p.num_work : max_units[dev];
   cfg.gridDim = dim3(static_cast<unsigned>(units * kCta), 1, 1);
   if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return FP8_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
+// Few rows (M <= 128): the GEMM streams B and its 128 x 256 tiles may not
+// fill the GPU.  With a workspace, such problems split K (plan_splits);
+// without one, narrow 128 x 64 tiles are used when 128 x 256 tiles would
+// leave more than half of the SMs idle and the narrow ones still fit in one
+// wave (measured on the Llama-2-70B projections at T <= 128: a second, mostly
+// empty wave of narrow tiles costs more than the idle SMs of the wide ones).
+bool few_wide_tiles(int64_t M, int64_t N) {
+  const int64_t wide = ((M + 127) / 128) * ((N + 255) / 256);
+  return M <= 128 && 2 * wide <= sm_count();
+}
+
 template <bool kAMN, bool kBMN, bool kOutF32, bool kAmax = false>
 int launch_pick(const GemmArgs& g, cudaStream_t s) {
-  // One 128-row tile covers M: single-CTA tiles; otherwise CTA pairs.  With
-  // so few rows the GEMM streams B, and every SM should get a share of it:
-  // narrow 128 x 64 tiles are used when 128 x 256 tiles would leave more than
-  // half of the SMs idle and the narrow ones still fit in one wave (measured on
-  // the Llama-2-70B projections at T <= 128: a second, mostly empty wave of
-  // narrow tiles costs more than the idle SMs of the wide ones).
   if (g.M <= 128) {
-    const int64_t wide = (g.N + 255) / 256, narrow = (g.N + 63) / 64;
-    if (!kBMN && 2 * wide < sm_count() && narrow <= sm_count())
+    const int64_t narrow = (g.N + 63) / 64;
+    if (!kBMN && g.workspace == nullptr && few_wide_tiles(g.M, g.N) && narrow <= sm_count())
       return launch_t<kTileNarrow, kAMN, false, kOutF32, kAmax>(g, s);
     return launch_t<kTileSingle, kAMN, kBMN, kOutF32, kAmax>(g, s);
   }
@@ -665,6 +808,15 @@ int launch_gemm(const GemmArgs& g, cudaStream_t s) {
     case 7: return launch_pick<true, true, true>(g, s);
     default: return FP8_ERR_UNSUPPORTED;   // MN-major A with K-major B: no pass uses it
   }
+}
+
+size_t gemm_workspace_bytes(const GemmArgs& g) {
+  if (!few_wide_tiles(g.M, g.N)) return 0;
+  const int tiles = static_cast<int>(((g.M + 127) / 128) * ((g.N + 255) / 256));
+  const int nkb = static_cast<int>((g.K + BK - 1) / BK);
+  int per = 0;
+  const int sp = plan_splits(g.M, tiles, nkb, &per);
+  return sp > 1 ? splitk_workspace_bytes(sp, g.M, g.N, tiles) : 0;
 }
 
 cudaError_t launch_selftest_wait(uint64_t timeout_ns) {

@@ -29,10 +29,17 @@ struct GemmArgs {
   bool d_fp32;
   float* d_amax;   // optional: receives max |D| (must be zeroed before the launch)
   int64_t M, N, K;
+  // optional split-K workspace (problems with few tiles); nullptr = never split
+  void* workspace = nullptr;
+  size_t workspace_bytes = 0;
 };
 
 // Returns 0 on success, an fp8_status_t code otherwise.
 int launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+// Bytes of split-K workspace launch_gemm would use for this problem when given
+// one (0: the problem is never split).  a/b/d pointers are not read.
+size_t gemm_workspace_bytes(const GemmArgs& g);
 
 cudaError_t launch_selftest_wait(uint64_t timeout_ns);
 int device_error_site(bool clear);

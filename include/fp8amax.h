@@ -150,6 +150,30 @@ fp8_status_t fp8_linear_bwd_dgrad_amax(const uint8_t *dy8, fp8_format_t fdy,
                                        void *dx, fp8_dtype_t dx_dtype, float *dx_amax,
                                        void *stream);
 
+/*
+ * fp8_linear_fwd for few tokens (T <= 64, e.g. decode-sized inference calls),
+ * where the GEMM streams the weights and one tile per 128 x 256 block of Y
+ * leaves SMs idle: with a caller-provided workspace a long K dimension is
+ * split across more CTAs, each writing an fp32 partial to the workspace, and
+ * the last CTA of each tile adds the partials in a fixed order (deterministic)
+ * before the unscale and the single rounding.  Results equal fp8_linear_fwd's
+ * within the GEMM tolerance (the fp32 summation order differs); shapes that do
+ * not split run exactly as fp8_linear_fwd.
+ *   fp8_linear_fwd_workspace_size(T, in, out) returns the bytes needed (0
+ *   when the problem is not split; then `workspace` may be NULL).  Needs a
+ *   current sm_100 device; returns 0 for invalid shapes.
+ *   workspace  device memory of at least that many bytes, 256-byte aligned,
+ *              owned by the caller; its contents on entry do not matter.
+ *              Two calls that share a workspace must not overlap on the GPU.
+ * FP8_ERR_INVALID_ARGUMENT when the workspace is too small.
+ */
+size_t fp8_linear_fwd_workspace_size(int64_t T, int64_t in, int64_t out);
+
+fp8_status_t fp8_linear_fwd_ws(const uint8_t *x8, fp8_format_t fx, const int32_t *bias_x,
+                               const uint8_t *w8, fp8_format_t fw, const int32_t *bias_w,
+                               int64_t T, int64_t in, int64_t out, void *y, fp8_dtype_t y_dtype,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *fp8_status_string(fp8_status_t status);
 

@@ -292,3 +292,60 @@ def test_bias_update_every_k_and_fixed_bias():
         ref, absref = oracle.linear(oracle.FWD, u8(layer.x8), E4, held[0], u8(layer.w8), E4,
                                     held[1], T, In, Out)
         assert_gemm_close(to_f64(layer.y), ref, absref, "every-3 fwd step %d" % step)
+
+
+@pytest.mark.parametrize("T", [1, 16, 33, 64, 77])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_split_k_few_tokens(T, out_dtype):
+    """Few-token forward with the split-K workspace: full oracle comparison on
+    a shape whose K splits (T <= 64), deterministic across calls; T = 77 runs
+    unsplit through the same entry point."""
+    In, Out = 12288, 512                     # 2 tiles of 128 x 256, 96 k-blocks
+    x, w, _ = _inputs(T, In, Out, seed=500 + T)
+    Q = _passes(x, w, None)
+    qx, bx, rqx, rbx, fx = Q["x"]
+    qw, bw, rqw, rbw, fw = Q["w"]
+    need = fp8.fp8_linear_fwd_workspace_size(T, In, Out)
+    assert (need > 0) == (T <= 64)
+    y1 = fp8.fp8_linear_fwd_ws(qx, fx, bx, qw, fw, bw, out_dtype=out_dtype)
+    y2 = fp8.fp8_linear_fwd_ws(qx, fx, bx, qw, fw, bw, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    ref, absref = oracle.linear(oracle.FWD, rqx, fx, rbx, rqw, fw, rbw, T, In, Out)
+    assert_gemm_close(to_f64(y1), ref, absref, "split-K T=%d" % T)
+
+
+@pytest.mark.parametrize("li", [3])
+def test_split_k_decode_llama70b(li):
+    """Decode-sized T on the Llama-2-70B down projection (the one that
+    splits: 32 wide tiles, K = 28672), sampled against the oracle."""
+    cfg = workloads.C3
+    lin = cfg.linears[li]
+    T = 16
+    x, w, _ = workloads.linear_inputs(3, li)
+    x = x[:T].contiguous()
+    Q = _passes(x, w, None)
+    qx, bx, rqx, rbx, fx = Q["x"]
+    qw, bw, rqw, rbw, fw = Q["w"]
+    assert fp8.fp8_linear_fwd_workspace_size(T, lin.in_features, lin.out_features) > 0
+    y = fp8.fp8_linear_fwd_ws(qx, fx, bx, qw, fw, bw)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(li)
+    rows = np.repeat(np.arange(T), 64)
+    cols = rng.integers(0, lin.out_features, rows.size)
+    ref, absref = oracle.linear_entries(oracle.FWD, rqx, fx, rbx, rqw, fw, rbw, T,
+                                        lin.in_features, lin.out_features, rows, cols)
+    assert_gemm_close(to_f64(y)[rows, cols], ref, absref, "decode %s" % lin.name)
+
+
+def test_split_k_workspace_errors():
+    T, In, Out = 8, 12288, 512
+    x8 = torch.zeros((T, In), dtype=torch.uint8, device=DEV)
+    w8 = torch.zeros((Out, In), dtype=torch.uint8, device=DEV)
+    b = torch.zeros(1, dtype=torch.int32, device=DEV)
+    small = torch.empty(256, dtype=torch.uint8, device=DEV)
+    with pytest.raises(fp8.Fp8Error) as e:
+        fp8.fp8_linear_fwd_ws(x8, E4, b, w8, E4, b, workspace=small)
+    assert e.value.status == 1
+    # a problem that does not split needs no workspace
+    assert fp8.fp8_linear_fwd_workspace_size(4096, 1024, 4096) == 0
