@@ -233,6 +233,30 @@ def fp8_linear_fwd_ws(x8, fx, bias_x, w8, fw, bias_w, out=None, out_dtype=torch.
     return out
 
 
+def fp8_linear_fwd_noalloc(x8, fx, bias_x, w8, fw, bias_w, out, stream=None):
+    """fp8_linear_fwd_ws without a workspace or any allocation: for callers
+    that may not allocate device memory when they run a forward.  `out` must
+    be given; the split-K scratch is the library's own 16 MiB array per GPU
+    (calls that overlap on the GPU must be serialised by the caller)."""
+    L = lib()
+    f = L.fp8_linear_fwd_noalloc
+    if f.argtypes is None:
+        c = ctypes
+        f.argtypes = [c.c_void_p, c.c_int, c.c_void_p, c.c_void_p, c.c_int, c.c_void_p,
+                      c.c_int64, c.c_int64, c.c_int64, c.c_void_p, c.c_int, c.c_void_p]
+        f.restype = c.c_int
+    T, in_ = x8.shape
+    out_ = w8.shape[0]
+    _need_cuda(x8, bias_x, w8, bias_w, out)
+    if tuple(out.shape) != (T, out_) or out.dtype not in _OUT:
+        raise ValueError("output must be [T, out] of bfloat16/float32")
+    s = stream if stream is not None else _stream_ptr(bias_x)
+    _check("fp8_linear_fwd_noalloc", f(_ptr(x8), int(fx), _ptr(bias_x), _ptr(w8), int(fw),
+                                       _ptr(bias_w), int(T), int(in_), int(out_), _ptr(out),
+                                       _OUT[out.dtype], ctypes.c_void_p(s)))
+    return out
+
+
 def fp8_linear_bwd_dgrad(dy8, fdy, bias_dy, w8, fw, bias_w, out=None, out_dtype=torch.bfloat16,
                          amax=False):
     """dX [T,in] = (dY8 [T,out] . W8 [out,in]) * 2^-(bias_dy + bias_w).
@@ -273,6 +297,6 @@ __all__ = [
     "E4M3", "E5M2", "BF16", "FP32", "FMT_MAX", "Fp8Error", "lib", "declared_entry_points",
     "fp8_status_string", "fp8_amax", "fp8_compute_bias", "fp8_cast_scaled", "fp8_quantize",
     "fp8_linear_fwd", "fp8_linear_bwd_dgrad", "fp8_linear_bwd_wgrad", "fp8_device_error",
-    "fp8_linear_fwd_ws", "fp8_linear_fwd_workspace_size",
+    "fp8_linear_fwd_ws", "fp8_linear_fwd_workspace_size", "fp8_linear_fwd_noalloc",
     "fp8_selftest_bounded_wait", "Fp8AmaxLinear",
 ]

@@ -264,6 +264,30 @@ fp8_status_t fp8_linear_fwd_ws(const uint8_t* x8, fp8_format_t fx, const int32_t
   return static_cast<fp8_status_t>(launch_gemm(g, as_stream(stream)));
 }
 
+fp8_status_t fp8_linear_fwd_noalloc(const uint8_t* x8, fp8_format_t fx, const int32_t* bias_x,
+                                    const uint8_t* w8, fp8_format_t fw, const int32_t* bias_w,
+                                    int64_t T, int64_t in, int64_t out, void* y,
+                                    fp8_dtype_t y_dtype, void* stream) {
+  if (fp8_status_t st = check_linear(x8, true, fx, bias_x, w8, false, fw, bias_w, T, in, out, y,
+                                     true, y_dtype))
+    return st;
+  if (fp8_status_t st = check_device()) return st;
+  if (T == 0) return FP8_OK;
+  GemmArgs g = {};
+  g.a = x8;
+  g.b = w8;
+  g.a_fmt = fx;
+  g.b_fmt = fw;
+  g.bias_a = bias_x;
+  g.bias_b = bias_w;
+  g.d = y;
+  g.d_fp32 = y_dtype == FP8_DTYPE_FP32;
+  g.M = T;
+  g.N = out;
+  g.K = in;
+  return static_cast<fp8_status_t>(launch_gemm_noalloc(g, as_stream(stream)));
+}
+
 fp8_status_t fp8_device_error(int clear, int32_t* where) {
   if (fp8_status_t st = check_device()) return st;
   const int site = device_error_site(clear != 0);

@@ -819,6 +819,44 @@ size_t gemm_workspace_bytes(const GemmArgs& g) {
   return sp > 1 ? splitk_workspace_bytes(sp, g.M, g.N, tiles) : 0;
 }
 
+// ----------------------------------------------------------------------------
+// Forward GEMM that allocates nothing (fp8_linear_fwd_noalloc).
+//
+// Some callers cannot allocate device memory at the point where they run a
+// forward: code inside a region that must not call cudaMalloc (an allocator
+// that is locked, a pre-sized memory pool that may not grow, a serving loop
+// that forbids allocation on its hot path), or plain C callers with no device
+// allocator of their own.  For them the split-K scratch lives in the array
+// below, which every GPU that loads this library holds until the process
+// exits.  Host code may not use the array's name as a device address: it is
+// looked up once per device with cudaGetSymbolAddress, with that device
+// current, on the first call made there.
+// ----------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;     // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+int launch_gemm_noalloc(GemmArgs g, cudaStream_t s) {
+  static void* scratch_addr[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
+  if (scratch_addr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return FP8_ERR_CUDA;
+    scratch_addr[dev] = ptr;
+  }
+  const size_t need = gemm_workspace_bytes(g);
+  if (need > kNoAllocScratchBytes) return FP8_ERR_UNSUPPORTED;
+  if (need > 0) {
+    // the split counters the kernel needs at zero are cleared by launch_gemm
+    // (a memset inside the array) before every launch; the fp32 partials are
+    // always written before they are read
+    g.workspace = scratch_addr[dev];
+    g.workspace_bytes = kNoAllocScratchBytes;
+  }
+  return launch_gemm(g, s);
+}
+
 cudaError_t launch_selftest_wait(uint64_t timeout_ns) {
   selftest_wait_kernel<<<1, 32>>>(timeout_ns);
   return cudaGetLastError();

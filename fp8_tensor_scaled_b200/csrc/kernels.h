@@ -41,6 +41,10 @@ int launch_gemm(const GemmArgs& g, cudaStream_t s);
 // one (0: the problem is never split).  a/b/d pointers are not read.
 size_t gemm_workspace_bytes(const GemmArgs& g);
 
+// launch_gemm with the split-K scratch taken from a static device array
+// instead of a caller workspace (FP8_ERR_UNSUPPORTED beyond its 16 MiB).
+int launch_gemm_noalloc(GemmArgs g, cudaStream_t s);
+
 cudaError_t launch_selftest_wait(uint64_t timeout_ns);
 int device_error_site(bool clear);
 

@@ -174,6 +174,30 @@ fp8_status_t fp8_linear_fwd_ws(const uint8_t *x8, fp8_format_t fx, const int32_t
                                int64_t T, int64_t in, int64_t out, void *y, fp8_dtype_t y_dtype,
                                void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * fp8_linear_fwd_ws for callers that cannot allocate device memory when they
+ * run a forward (an allocator that must not be entered there, a fixed memory
+ * pool, a serving loop that forbids allocation, a C program with no device
+ * allocator).  The paper has no counterpart: this is a packaging of the same
+ * forward.  Same arguments and results as fp8_linear_fwd_ws without the
+ * workspace: the split-K scratch is a 16 MiB array inside the library that
+ * every GPU which loads the library holds until the process exits.
+ *   - The first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Nothing is allocated, by this call or below it.
+ *   - A problem whose split-K scratch would exceed 16 MiB (only possible for
+ *     T <= 64 with very wide outputs) returns FP8_ERR_UNSUPPORTED; problems
+ *     that do not split use no scratch at all.
+ *   - All calls share the one array and it keeps the last call's contents:
+ *     calls that overlap on the GPU (different streams, no ordering between
+ *     them) race on it and must be serialised by the caller.
+ */
+fp8_status_t fp8_linear_fwd_noalloc(const uint8_t *x8, fp8_format_t fx, const int32_t *bias_x,
+                                    const uint8_t *w8, fp8_format_t fw, const int32_t *bias_w,
+                                    int64_t T, int64_t in, int64_t out,
+                                    void *y, fp8_dtype_t y_dtype, void *stream);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char *fp8_status_string(fp8_status_t status);
 
