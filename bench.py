@@ -330,86 +330,111 @@ def run_e2e(args, wl, device, world):
 
 
 # ------------------------------------------------------------------ CPU oracle
-def oracle_sample(cid, seconds=15.0):
-    """Time the CPU oracle on a bounded sample of one step and extrapolate.
+class OracleSample:
+    """The CPU oracle timed on a bounded sample of one step, extrapolated.
 
     Sample: for every projection and pass, an 8 x `cols` block of output
     elements of the fp64 oracle matmul (full K each), plus amax + bias + cast of
-    the first 2^22 elements of each of the step's input tensors.  The oracle's
-    cost is linear in output elements x K and in elements cast, so the whole
-    step's CPU time is extrapolated by FLOPs and by elements.  `cols` is sized
-    for roughly `seconds` of CPU time at the oracle's measured rate."""
-    import numpy as np
+    2^22 elements of each of the step's input tensors.  The oracle's cost is
+    linear in output elements x K and in elements cast, so the whole step's CPU
+    time is extrapolated by FLOPs and by elements.  Operands (seeded FP8 codes
+    and BF16 values of the real shapes) are drawn once; `cols` is sized for
+    roughly `seconds` of CPU time at the oracle's measured rate."""
 
-    import oracle
-    cfg = workloads.CONFIGS[cid]
-    rng = np.random.default_rng(1)
-    g = torch.Generator().manual_seed(1)
-    n_q = 1 << 22
-    t_quant, n_quant_done, n_quant_total = 0.0, 0, 0
-    for lin in cfg.linears:
-        for shape in ((cfg.tokens, lin.in_features), (lin.out_features, lin.in_features),
-                      (cfg.tokens, lin.out_features)):
-            n_quant_total += shape[0] * shape[1]
-            x = torch.randn(min(n_q, shape[0] * shape[1]), generator=g).to(torch.bfloat16)
-            t0 = time.perf_counter()
-            oracle.quantize(x, 0, 0)
-            t_quant += time.perf_counter() - t0
-            n_quant_done += x.numel()
+    def __init__(self, cid, seconds=15.0):
+        import numpy as np
 
-    def block(rows, cols):
+        import oracle
+        self.oracle = oracle
+        self.cfg = cfg = workloads.CONFIGS[cid]
+        rng = np.random.default_rng(1)
+        g = torch.Generator().manual_seed(1)
+        T = cfg.tokens
+        self.ops = []
+        for lin in cfg.linears:
+            In, Out = lin.in_features, lin.out_features
+            X = rng.integers(0, 120, (T, In), dtype=np.uint8)
+            W = rng.integers(0, 120, (Out, In), dtype=np.uint8)
+            dY = rng.integers(0, 120, (T, Out), dtype=np.uint8)
+            self.ops.append((lin, X, W, dY))
+        self.quant_in = []
+        self.n_quant_total = 0
+        for lin in cfg.linears:
+            for shape in ((T, lin.in_features), (lin.out_features, lin.in_features),
+                          (T, lin.out_features)):
+                self.n_quant_total += shape[0] * shape[1]
+                n = min(1 << 22, shape[0] * shape[1])
+                self.quant_in.append(torch.randn(n, generator=g).to(torch.bfloat16))
+        self.set_seconds(seconds)
+
+    def set_seconds(self, seconds):
+        import numpy as np
+        lin0, X, W, _ = self.ops[0]
+        r, c = self._block(8, 64)
+        t0 = time.perf_counter()
+        self.oracle.linear_entries(self.oracle.FWD, X, 0, 0, W, 0, 0, self.cfg.tokens,
+                                   lin0.in_features, lin0.out_features, r, c)
+        rate = 2.0 * r.size * lin0.in_features / (time.perf_counter() - t0)     # FLOP/s
+        k_sum = sum(l.in_features + l.out_features + self.cfg.tokens for l in self.cfg.linears)
+        self.cols = int(max(16, min(4096, seconds * rate / (2.0 * 8 * k_sum))))
+
+    @staticmethod
+    def _block(rows, cols):
+        import numpy as np
         r, c = np.meshgrid(np.arange(rows), np.arange(cols), indexing="ij")
         return r.ravel(), c.ravel()
 
-    # measure the rate on a small block first, then size the sample to `seconds`
-    T = cfg.tokens
-    lin0 = cfg.linears[0]
-    X = rng.integers(0, 120, (T, lin0.in_features), dtype=np.uint8)
-    W = rng.integers(0, 120, (lin0.out_features, lin0.in_features), dtype=np.uint8)
-    r, c = block(8, 64)
-    t0 = time.perf_counter()
-    oracle.linear_entries(oracle.FWD, X, 0, 0, W, 0, 0, T, lin0.in_features, lin0.out_features,
-                          r, c)
-    rate = 2.0 * r.size * lin0.in_features / (time.perf_counter() - t0)       # FLOP/s
-    k_sum = sum(l.in_features + l.out_features + T for l in cfg.linears)
-    cols = int(max(16, min(4096, seconds * rate / (2.0 * 8 * k_sum))))
-
-    t_gemm, f_gemm_done = 0.0, 0
-    for lin in cfg.linears:
-        In, Out = lin.in_features, lin.out_features
-        X = rng.integers(0, 120, (T, In), dtype=np.uint8)
-        W = rng.integers(0, 120, (Out, In), dtype=np.uint8)
-        dY = rng.integers(0, 120, (T, Out), dtype=np.uint8)
-        for p, A, fa, B, K, ncols in ((oracle.FWD, X, 0, W, In, Out), (oracle.DGRAD, dY, 1, W, Out, In),
-                                      (oracle.WGRAD, dY, 1, X, T, In)):
-            r, c = block(8, min(cols, ncols))
+    def run(self):
+        o = self.oracle
+        T = self.cfg.tokens
+        t_quant, n_quant_done = 0.0, 0
+        for x in self.quant_in:
             t0 = time.perf_counter()
-            oracle.linear_entries(p, A, fa, 0, B, 0, 0, T, In, Out, r, c)
-            t_gemm += time.perf_counter() - t0
-            f_gemm_done += 2 * r.size * K
-    flops = cfg.flops_per_step()
-    est_step = t_gemm * flops / f_gemm_done + t_quant * n_quant_total / n_quant_done
-    sample = ("CPU oracle on an 8 x %d block of output elements (full K) of each of the %d "
-              "matmuls of the step, plus amax+bias+cast of 2^22 elements of each of the %d "
-              "input tensors; whole-step time extrapolated by FLOPs and elements"
-              % (cols, 3 * len(cfg.linears), 3 * len(cfg.linears)))
-    return {"value": flops / est_step / 1e12, "unit": UNIT, "cores": oracle.num_threads(),
-            "kind": "oracle", "sample": sample, "sample_seconds": round(t_gemm + t_quant, 3),
-            "est_step_seconds": round(est_step, 1)}
+            o.quantize(x, 0, 0)
+            t_quant += time.perf_counter() - t0
+            n_quant_done += x.numel()
+        t_gemm, f_gemm_done = 0.0, 0
+        for lin, X, W, dY in self.ops:
+            In, Out = lin.in_features, lin.out_features
+            for p, A, fa, B, K, ncols in ((o.FWD, X, 0, W, In, Out), (o.DGRAD, dY, 1, W, Out, In),
+                                          (o.WGRAD, dY, 1, X, T, In)):
+                r, c = self._block(8, min(self.cols, ncols))
+                t0 = time.perf_counter()
+                o.linear_entries(p, A, fa, 0, B, 0, 0, T, In, Out, r, c)
+                t_gemm += time.perf_counter() - t0
+                f_gemm_done += 2 * r.size * K
+        flops = self.cfg.flops_per_step()
+        est_step = (t_gemm * flops / f_gemm_done
+                    + t_quant * self.n_quant_total / n_quant_done)
+        n = 3 * len(self.cfg.linears)
+        sample = ("CPU oracle on an 8 x %d block of output elements (full K) of each of the %d "
+                  "matmuls of the step, plus amax+bias+cast of 2^22 elements of each of the %d "
+                  "input tensors; whole-step time extrapolated by FLOPs and elements"
+                  % (self.cols, n, n))
+        return {"value": flops / est_step / 1e12, "unit": UNIT, "cores": o.num_threads(),
+                "kind": "oracle", "sample": sample, "sample_seconds": round(t_gemm + t_quant, 3),
+                "est_step_seconds": round(est_step, 1)}
+
+
+def oracle_sample(cid, seconds=15.0):
+    return OracleSample(cid, seconds).run()
 
 
 def run_reference(args, world, rank):
-    """The reference arm: the CPU oracle, timed as it stands (rank 0 only)."""
+    """The reference arm: the CPU oracle, timed as it stands (rank 0 only).
+    Every step is a bounded sample of the step (OracleSample), sized so that
+    the whole --warmup + --steps run stays within a few minutes."""
     if rank != 0:
         return 0
     cid = int(args.workload[1:])
+    per_step = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
+    sampler = OracleSample(cid, per_step)
     for _ in range(args.warmup):
-        oracle_sample(cid, args.cpu_seconds)
-    vals, secs = [], []
+        sampler.run()
+    vals, r = [], None
     for _ in range(args.steps):
-        r = oracle_sample(cid, args.cpu_seconds)
+        r = sampler.run()
         vals.append(r["value"])
-        secs.append(r["sample_seconds"])
     v = statistics.median(vals)
     cfg = workloads.CONFIGS[cid]
     line = {

@@ -38,18 +38,22 @@ def _worker(rank, world, port, q):
     bench.barrier(w)
     calls = []
 
-    def fake_sample(cid, seconds=15.0):
-        calls.append(cid)
-        return {"value": 1.5e-3, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                "sample": "fake", "sample_seconds": 0.0, "est_step_seconds": 1.0}
+    class FakeSample:
+        def __init__(self, cid, seconds=15.0):
+            calls.append(("init", cid))
 
-    bench.oracle_sample = fake_sample
+        def run(self):
+            calls.append("run")
+            return {"value": 1.5e-3, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                    "sample": "fake", "sample_seconds": 0.0, "est_step_seconds": 1.0}
+
+    bench.OracleSample = FakeSample
     out = io.StringIO()
     with redirect_stdout(out):
         rc = bench.run_reference(args, w, r)
     bench.barrier(w)
     dist.destroy_process_group()
-    q.put((r, m, rc, out.getvalue(), len(calls)))
+    q.put((r, m, rc, out.getvalue(), calls.count("run")))
 
 
 def test_two_ranks_gloo():
