@@ -60,6 +60,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-overlap", action="store_true",
                     help="run each projection's quantization and GEMMs strictly in order")
+    ap.add_argument("--graph", action="store_true",
+                    help="time the step as CUDA-graph replays (one host call per step); the "
+                         "per-kernel split still comes from an eager pass of the same steps")
     ap.add_argument("--bias-every", type=int, default=1,
                     help="recompute amax/bias every k steps (1 = FP8-AMAX every step, the "
                          "default; k > 1 casts with the stored bias in between)")
@@ -254,6 +257,23 @@ def run_fp8(args, world, rank, local):
     res = dict(ms=ms, ms_local=ms_local, quant_ms=quant_ms, gemm_ms=gemm_ms,
                per_linear_gemm_ms=per_linear_gemm_ms, clocks=clocks, wl=wl,
                quant_bytes=quant_bytes)
+    if args.graph:
+        wl.stepper.capture(wl.inputs)
+        for _ in range(max(3, args.warmup)):
+            wl.stepper.replay()
+        torch.cuda.synchronize(device)
+        barrier(world)
+        sampler = ClockSampler(local)
+        time.sleep(0.3)
+        start.record(stream)
+        for _ in range(args.steps):
+            wl.stepper.replay()
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        res["clocks"] = sampler.stop()
+        barrier(world)
+        res["ms_eager"] = ms
+        res["ms"] = max_over_ranks(world, start.elapsed_time(end), device)
 
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, wl, device, world)
@@ -502,6 +522,7 @@ def main():
         "data": "synthetic", "config": config_dict(wl.cfg, world),
         "gemm_tflops": round(gemm_tflops, 2), "quant_gbs": round(quant_gbs, 1),
         "overlap": not args.no_overlap, "bias_update_every": args.bias_every,
+        "launch": "cuda-graph" if args.graph else "eager",
         "per_linear_gemm_ms": [round(x, 4) for x in r["per_linear_gemm_ms"]],
         "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 2), "peak": round(fp8_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_tflops / fp8_peak, 4),
@@ -518,6 +539,8 @@ def main():
         "clocks": r["clocks"],
         "gpu_launches": wl.kernels_per_step * steps,
     }
+    if "ms_eager" in r:
+        line["ms_per_step_eager"] = round(r["ms_eager"] / steps, 4)
     if "e2e" in r:
         e = r["e2e"]
         line["e2e"] = {"value": round(total_flops / (e["ms_per_step"] * 1e-3) / 1e12, 2),

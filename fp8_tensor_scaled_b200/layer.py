@@ -101,6 +101,9 @@ class Fp8AmaxStep:
     energy of its work rather than by the order of it.)
 
     ``step(inputs)``            inputs already on the device: [(x, w, dy), ...]
+    ``capture(inputs)`` / ``replay()``  the same step recorded once into a CUDA
+        graph (on these input and output buffers) and replayed with a single
+        host call: no per-kernel launch cost, which matters for small layers.
     ``step_from_host(h_in, d_in, h_out)``  the same step from pinned host tensors:
         copies in on one copy stream, copies of each linear's Y, dX, dW out on
         another as soon as its GEMMs finish, so transfers in both directions
@@ -157,6 +160,28 @@ class Fp8AmaxStep:
             if timing is not None:
                 timing["g"][i][1].record(main)
             self.g_done[i].record(main)
+
+    def capture(self, inputs):
+        """Record one step into a CUDA graph.  The graph replays the exact
+        kernels recorded, so the per-step host decisions must be fixed: every
+        linear recomputes its biases every step (bias_update_every == 1) or
+        uses fixed biases."""
+        if any(l.fixed is None and l.every != 1 for l in self.linears):
+            raise ValueError("a captured step needs bias_update_every == 1 or fixed biases")
+        dev = self.device
+        warm = torch.cuda.Stream(dev)
+        warm.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(warm):          # first calls set up per-device state
+            self.step(inputs)
+        torch.cuda.current_stream(dev).wait_stream(warm)
+        torch.cuda.synchronize(dev)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step(inputs)
+        return self.graph
+
+    def replay(self):
+        self.graph.replay()
 
     def step_from_host(self, host_inputs, device_inputs, host_outputs):
         main = torch.cuda.current_stream(self.device)

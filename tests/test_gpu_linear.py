@@ -349,3 +349,31 @@ def test_split_k_workspace_errors():
     assert e.value.status == 1
     # a problem that does not split needs no workspace
     assert fp8.fp8_linear_fwd_workspace_size(4096, 1024, 4096) == 0
+
+
+def test_step_graph_replay_matches_eager():
+    """A multi-linear step recorded into a CUDA graph replays the same
+    kernels: outputs, biases and codes equal the eager step's bit for bit."""
+    from fp8_tensor_scaled_b200.layer import Fp8AmaxStep
+    shapes = [(256, 384, 512), (256, 512, 256)]
+    inputs, eager_l, graph_l = [], [], []
+    for i, (T, In, Out) in enumerate(shapes):
+        x, w, dy = _inputs(T, In, Out, seed=900 + i)
+        inputs.append((x.to(DEV), w.to(DEV), dy.to(DEV)))
+        eager_l.append(fp8.Fp8AmaxLinear(T, In, Out, DEV))
+        graph_l.append(fp8.Fp8AmaxLinear(T, In, Out, DEV))
+    eager = Fp8AmaxStep(eager_l)
+    graph = Fp8AmaxStep(graph_l)
+    graph.capture(inputs)
+    for _ in range(2):
+        eager.step(inputs)
+        graph.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(eager_l, graph_l):
+        for name in ("y", "dx", "dw", "x8", "w8", "dy8", "bias", "amax"):
+            assert torch.equal(getattr(a, name), getattr(b, name)), name
+    with pytest.raises(ValueError):
+        Fp8AmaxStep([fp8.Fp8AmaxLinear(16, 16, 16, DEV, bias_update_every=2)]).capture(
+            [(inputs[0][0][:16, :16].contiguous(), inputs[0][1][:16, :16].contiguous(),
+              inputs[0][2][:16, :16].contiguous())])
+
