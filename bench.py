@@ -346,7 +346,36 @@ def run_e2e(args, wl, device, world):
     b.record(stream)
     b.synchronize()
     ms = max_over_ranks(world, a.elapsed_time(b), device) / args.e2e_steps
-    return {"ms_per_step": ms, "h2d": h2d, "d2h": d2h}
+
+    # The copy floor of this step: the same copies with no compute, in each
+    # direction alone and in both at once (copy engines, pinned host memory).
+    def copies(up, down):
+        s_up, s_down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        s_up.wait_stream(stream)
+        s_down.wait_stream(stream)
+        if up:
+            with torch.cuda.stream(s_up):
+                for hs, ds in zip(host_in, wl.inputs):
+                    for h, d in zip(hs, ds):
+                        d.copy_(h, non_blocking=True)
+        if down:
+            with torch.cuda.stream(s_down):
+                for lin, hs in zip(wl.layers, host_out):
+                    for h, d in zip(hs, (lin.y, lin.dx, lin.dw)):
+                        h.copy_(d, non_blocking=True)
+        stream.wait_stream(s_up)
+        stream.wait_stream(s_down)
+
+    floor = {}
+    for name, up, down in (("h2d", True, False), ("d2h", False, True), ("both", True, True)):
+        copies(up, down)
+        torch.cuda.synchronize(device)
+        a.record(stream)
+        copies(up, down)
+        b.record(stream)
+        b.synchronize()
+        floor[name] = max_over_ranks(world, a.elapsed_time(b), device)
+    return {"ms_per_step": ms, "h2d": h2d, "d2h": d2h, "copy_ms": floor}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -545,7 +574,14 @@ def main():
         e = r["e2e"]
         line["e2e"] = {"value": round(total_flops / (e["ms_per_step"] * 1e-3) / 1e12, 2),
                        "unit": UNIT, "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
-                       "ms_per_step": round(e["ms_per_step"], 3)}
+                       "ms_per_step": round(e["ms_per_step"], 3),
+                       "copy_floor": {"bound": "pcie",
+                                      "h2d_gbs": round(e["h2d"] / e["copy_ms"]["h2d"] / 1e6, 1),
+                                      "d2h_gbs": round(e["d2h"] / e["copy_ms"]["d2h"] / 1e6, 1),
+                                      "both_ms": round(e["copy_ms"]["both"], 3),
+                                      "frac": round(e["copy_ms"]["both"] / e["ms_per_step"], 4),
+                                      "note": "the step's copies alone, both directions at "
+                                              "once, no compute; frac = that time / e2e time"}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = oracle_sample(int(args.workload[1:]), args.cpu_seconds)
         line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}

@@ -64,6 +64,8 @@ def lib():
                                       vp, vp],
         "fp8_linear_fwd_ws": [vp, c.c_int, vp, vp, c.c_int, vp, i64, i64, i64, vp, c.c_int, vp,
                               sz, vp],
+        "fp8_linear_bwd_wgrad_ws": [vp, c.c_int, vp, vp, c.c_int, vp, i64, i64, i64, vp, c.c_int,
+                                    vp, sz, vp],
         "fp8_device_error": [c.c_int, vp],
         "fp8_selftest_bounded_wait": [u64],
         "fp8_abi_version": [],
@@ -76,6 +78,8 @@ def lib():
     L.fp8_status_string.restype = c.c_char_p
     L.fp8_linear_fwd_workspace_size.argtypes = [i64, i64, i64]
     L.fp8_linear_fwd_workspace_size.restype = sz
+    L.fp8_linear_bwd_wgrad_workspace_size.argtypes = [i64, i64, i64]
+    L.fp8_linear_bwd_wgrad_workspace_size.restype = sz
     _lib = L
     return L
 
@@ -270,6 +274,55 @@ def fp8_linear_bwd_dgrad(dy8, fdy, bias_dy, w8, fw, bias_w, out=None, out_dtype=
                    (T, in_), out, out_dtype, amax)
 
 
+FWD, DGRAD, WGRAD = 0, 1, 2
+
+
+class _Plan(ctypes.Structure):
+    _fields_ = [("tile_m", ctypes.c_int32), ("tile_n", ctypes.c_int32),
+                ("ctas_per_tile", ctypes.c_int32), ("k_splits", ctypes.c_int32)]
+
+
+def fp8_linear_plan(pass_, T, in_, out_, with_workspace=False):
+    """The launch plan of one pass on the current device:
+    {"tile_m", "tile_n", "ctas_per_tile", "k_splits"}."""
+    L = lib()
+    f = L.fp8_linear_plan
+    f.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                  ctypes.POINTER(_Plan)]
+    f.restype = ctypes.c_int
+    p = _Plan()
+    _check("fp8_linear_plan", f(int(pass_), int(T), int(in_), int(out_), int(bool(with_workspace)),
+                                ctypes.byref(p)))
+    return {k: int(getattr(p, k)) for k, _ in _Plan._fields_}
+
+
+def fp8_linear_bwd_wgrad_workspace_size(T, in_, out_):
+    """Bytes of workspace fp8_linear_bwd_wgrad_ws splits K with (0: no split)."""
+    return int(lib().fp8_linear_bwd_wgrad_workspace_size(int(T), int(in_), int(out_)))
+
+
+def fp8_linear_bwd_wgrad_ws(dy8, fdy, bias_dy, x8, fx, bias_x, out=None,
+                            out_dtype=torch.bfloat16, workspace=None):
+    """fp8_linear_bwd_wgrad with a split-K workspace (allocated here through
+    torch when not given) for small weight gradients over many tokens."""
+    T, out_ = dy8.shape
+    in_ = x8.shape[1]
+    assert x8.shape[0] == T
+    _need_cuda(dy8, bias_dy, x8, bias_x, out, workspace)
+    dev = bias_dy.device
+    if out is None:
+        out = torch.empty((out_, in_), dtype=out_dtype, device=dev)
+    need = fp8_linear_bwd_wgrad_workspace_size(T, in_, out_)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("fp8_linear_bwd_wgrad_ws", lib().fp8_linear_bwd_wgrad_ws(
+        _ptr(dy8), int(fdy), _ptr(bias_dy), _ptr(x8), int(fx), _ptr(bias_x), int(T), int(in_),
+        int(out_), _ptr(out), _OUT[out.dtype], _ptr(workspace), nbytes,
+        ctypes.c_void_p(_stream_ptr(bias_dy))))
+    return out
+
+
 def fp8_linear_bwd_wgrad(dy8, fdy, bias_dy, x8, fx, bias_x, out=None, out_dtype=torch.bfloat16):
     """dW [out,in] = (dY8 [T,out]^T . X8 [T,in]) * 2^-(bias_dy + bias_x)."""
     T, out_ = dy8.shape
@@ -298,5 +351,6 @@ __all__ = [
     "fp8_status_string", "fp8_amax", "fp8_compute_bias", "fp8_cast_scaled", "fp8_quantize",
     "fp8_linear_fwd", "fp8_linear_bwd_dgrad", "fp8_linear_bwd_wgrad", "fp8_device_error",
     "fp8_linear_fwd_ws", "fp8_linear_fwd_workspace_size", "fp8_linear_fwd_noalloc",
+    "fp8_linear_bwd_wgrad_ws", "fp8_linear_bwd_wgrad_workspace_size", "fp8_linear_plan",
     "fp8_selftest_bounded_wait", "Fp8AmaxLinear",
 ]

@@ -288,6 +288,78 @@ fp8_status_t fp8_linear_fwd_noalloc(const uint8_t* x8, fp8_format_t fx, const in
   return static_cast<fp8_status_t>(launch_gemm_noalloc(g, as_stream(stream)));
 }
 
+size_t fp8_linear_bwd_wgrad_workspace_size(int64_t T, int64_t in, int64_t out) {
+  if (T <= 0 || in <= 0 || out <= 0 || check_device() != FP8_OK) return 0;
+  GemmArgs g = {};
+  g.M = out;
+  g.N = in;
+  g.K = T;
+  return gemm_workspace_bytes(g);
+}
+
+fp8_status_t fp8_linear_bwd_wgrad_ws(const uint8_t* dy8, fp8_format_t fdy, const int32_t* bias_dy,
+                                     const uint8_t* x8, fp8_format_t fx, const int32_t* bias_x,
+                                     int64_t T, int64_t in, int64_t out, void* dw,
+                                     fp8_dtype_t dw_dtype, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (fp8_status_t st = check_linear(dy8, true, fdy, bias_dy, x8, true, fx, bias_x, T, in, out, dw,
+                                     false, dw_dtype))
+    return st;
+  if (workspace_bytes > 0 && !workspace) return FP8_ERR_INVALID_ARGUMENT;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FP8_ERR_MISALIGNED;
+  if (fp8_status_t st = check_device()) return st;
+  if (T == 0) {
+    const size_t bytes = static_cast<size_t>(out) * static_cast<size_t>(in) *
+                         (dw_dtype == FP8_DTYPE_FP32 ? 4 : 2);
+    return from_cuda(cudaMemsetAsync(dw, 0, bytes, as_stream(stream)));
+  }
+  GemmArgs g = {};
+  g.a = dy8;
+  g.b = x8;
+  g.a_fmt = fdy;
+  g.b_fmt = fx;
+  g.a_mn_major = true;
+  g.b_mn_major = true;
+  g.bias_a = bias_dy;
+  g.bias_b = bias_x;
+  g.d = dw;
+  g.d_fp32 = dw_dtype == FP8_DTYPE_FP32;
+  g.M = out;
+  g.N = in;
+  g.K = T;
+  const size_t need = gemm_workspace_bytes(g);
+  if (need > 0) {
+    if (workspace_bytes < need) return FP8_ERR_INVALID_ARGUMENT;
+    g.workspace = workspace;
+    g.workspace_bytes = workspace_bytes;
+  }
+  return static_cast<fp8_status_t>(launch_gemm(g, as_stream(stream)));
+}
+
+fp8_status_t fp8_linear_plan(fp8_pass_t pass, int64_t T, int64_t in, int64_t out,
+                             int with_workspace, fp8_gemm_plan_t* plan) {
+  if (!plan || T < 0 || in < 0 || out < 0) return FP8_ERR_INVALID_ARGUMENT;
+  if (pass != FP8_PASS_FWD && pass != FP8_PASS_DGRAD && pass != FP8_PASS_WGRAD)
+    return FP8_ERR_INVALID_ARGUMENT;
+  if (fp8_status_t st = check_device()) return st;
+  GemmArgs g = {};
+  g.M = pass == FP8_PASS_WGRAD ? out : T;
+  g.N = pass == FP8_PASS_FWD ? out : in;
+  g.K = pass == FP8_PASS_FWD ? in : (pass == FP8_PASS_DGRAD ? out : T);
+  g.a_mn_major = pass == FP8_PASS_WGRAD;
+  g.b_mn_major = pass != FP8_PASS_FWD;
+  // the passes with a workspace entry point: fwd and wgrad
+  static unsigned char marker;
+  if (with_workspace && pass != FP8_PASS_DGRAD) g.workspace = &marker;
+  GemmPlan p = {};
+  gemm_plan(g, &p);
+  plan->tile_m = p.tile_m;
+  plan->tile_n = p.tile_n;
+  plan->ctas_per_tile = p.ctas_per_tile;
+  plan->k_splits = p.k_splits;
+  return FP8_OK;
+}
+
 fp8_status_t fp8_device_error(int clear, int32_t* where) {
   if (fp8_status_t st = check_device()) return st;
   const int site = device_error_site(clear != 0);

@@ -14,14 +14,16 @@
 //   Tiles of 256 x 256 are computed by a CTA pair (a cluster of two) with
 //   tcgen05.mma.cta_group::2 (M=256, N=256, K=32): CTA r holds rows
 //   [128r, 128r+128) of the A tile, rows [128r, 128r+128) of the B tile and of
-//   the accumulator.  Problems with M <= 128 use one CTA per 128 x 256 tile.
+//   the accumulator.  Problems with M <= 128 use one CTA per 128 x 256 tile;
+//   problems of many tiles use 256 x 512 tiles (two such MMAs per K step that
+//   share the A stage: a quarter less L2 traffic per FLOP).
 //   warp 0      TMA producer: 128 x 128-byte FP8 boxes with 128-byte swizzle
 //               (no multicast: each CTA loads its own halves) into a 6-stage
 //               shared-memory ring of 32 KB stages (4 x 48 KB for one CTA);
 //               the pair's copies complete on the leader's mbarrier, armed
 //               with the bytes of both CTAs.
 //   warp 1      TMEM allocator (512 columns = two 128 x 256 fp32 accumulators
-//               per CTA); in the leader, one thread issues the MMAs (four per
+//               per CTA, or one 128 x 512 for 256 x 512 tiles); in the leader, one thread issues the MMAs (four per
 //               stage) and tcgen05.commit, multicast to both CTAs' barriers,
 //               frees each stage and publishes each finished accumulator.
 //   warps 2-5   epilogue: tcgen05.ld 32x32b of the CTA's accumulator rows,
@@ -99,27 +101,43 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 //   kTileNarrow  one CTA computes a 128 x 64 tile (M=128, N=64), K-major B only:
 //                for few rows (decode-sized T) the GEMM streams the weights, and
 //                narrow tiles give every SM a share of them.
+//   kTileDouble  a CTA pair computes a 256 x 512 tile as two cta_group::2 MMAs
+//                (M=256, N=256) per K step that share the A stage: CTA r loads
+//                A rows [128r, +128) and B rows [128r, +128) and [256+128r, +128)
+//                of the tile.  A CTA moves 48 KB from L2 per 128 x 512 x 128
+//                block instead of 64 KB for two 128 x 256 blocks (a quarter
+//                less L2 -> shared memory traffic per FLOP), at the price of a
+//                single 512-column accumulator: the epilogue drains it in two
+//                256-column halves, and the next tile's MMAs into a half wait
+//                only for that half.
 constexpr int BK = 128;                 // K per stage: one 128-byte swizzle row of FP8
 constexpr int UK = 32;                  // K per tcgen05.mma of kind::f8f6f4
 constexpr uint32_t A_BYTES = 128 * BK;  // 16 KB: 128 rows of A per CTA
 constexpr int kThreads = 192;           // 6 warps
 
-enum TileKind : int { kTileSingle = 0, kTilePair = 1, kTileNarrow = 2 };
+enum TileKind : int { kTileSingle = 0, kTilePair = 1, kTileNarrow = 2, kTileDouble = 3 };
 
+// BN: tile columns; MMA_N: N of one tcgen05.mma; B_ROWS: B rows per CTA and stage.
 template <int kTile> struct Cfg;
 template <> struct Cfg<kTileSingle> {
-  static constexpr int CTAS = 1, BM = 128, BN = 256, B_ROWS = 256, STAGES = 4;
+  static constexpr int CTAS = 1, BM = 128, BN = 256, MMA_N = 256, B_ROWS = 256, STAGES = 4;
 };
 template <> struct Cfg<kTilePair> {
-  static constexpr int CTAS = 2, BM = 256, BN = 256, B_ROWS = 128, STAGES = 6;
+  static constexpr int CTAS = 2, BM = 256, BN = 256, MMA_N = 256, B_ROWS = 128, STAGES = 6;
 };
 template <> struct Cfg<kTileNarrow> {
-  static constexpr int CTAS = 1, BM = 128, BN = 64, B_ROWS = 64, STAGES = 8;
+  static constexpr int CTAS = 1, BM = 128, BN = 64, MMA_N = 64, B_ROWS = 64, STAGES = 8;
 };
+template <> struct Cfg<kTileDouble> {
+  static constexpr int CTAS = 2, BM = 256, BN = 512, MMA_N = 256, B_ROWS = 256, STAGES = 4;
+};
+constexpr uint32_t B_HALF_BYTES = 128 * BK;   // 16 KB: one 128-row B box
 template <int kTile> constexpr uint32_t b_bytes() { return Cfg<kTile>::B_ROWS * BK; }
 template <int kTile> constexpr uint32_t stage_bytes() { return A_BYTES + b_bytes<kTile>(); }
-// two fp32 accumulators of BN columns each
-template <int kTile> constexpr uint32_t tmem_cols() { return 2 * Cfg<kTile>::BN; }
+// two fp32 accumulators of BN columns each; the wide tile has one of 512
+template <int kTile> constexpr uint32_t tmem_cols() {
+  return kTile == kTileDouble ? 512u : 2u * Cfg<kTile>::BN;
+}
 template <int kTile> constexpr int num_bars() { return 2 * Cfg<kTile>::STAGES + 2 + 2 + 1; }
 template <int kTile> constexpr size_t smem_bytes() {
   return 1024 + Cfg<kTile>::STAGES * stage_bytes<kTile>() + num_bars<kTile>() * 8 + 16;
@@ -131,13 +149,11 @@ struct Params {
   int group_n;
   // Split K: each tile's K range is cut into `splits` ranges of kb_per_split
   // k-blocks; work unit u is (tile u / splits, range u % splits).  With
-  // splits > 1 every unit writes its fp32 partial to ws[range][M][N], and for
-  // each 32-row quarter of a tile the last unit to finish it (counted in
-  // counters[tile * 4 + quarter]) adds the partials in range order and runs
-  // the epilogue on those rows.
+  // splits > 1 every unit writes its raw fp32 partial to ws[range][M][N] and
+  // splitk_reduce_kernel, launched next on the same stream, adds the partials
+  // in range order and runs the epilogue.
   int splits, kb_per_split, num_work;
   float* ws;
-  uint32_t* counters;
   uint32_t idesc;
   const int32_t* bias_a;
   const int32_t* bias_b;
@@ -272,7 +288,11 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   constexpr uint32_t STAGE_BYTES = stage_bytes<kTile>();
   constexpr uint32_t TMEM_COLS = tmem_cols<kTile>();
   constexpr int kNumBars = num_bars<kTile>();
+  // wide tile: one accumulator in two halves; tempty_bar(h) frees half h
+  constexpr bool kDbl = kTile == kTileDouble;
+  constexpr int kHalves = kDbl ? 2 : 1;
   static_assert(kTile != kTileNarrow || !kBMN, "narrow tiles take a K-major B only");
+  static_assert(TMEM_COLS <= 512, "tensor memory holds 512 columns");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -342,6 +362,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       tile_coords(t, p, mb, nb);
       const int a_row = mb * C::BM + static_cast<int>(rank) * 128;
       const int b_row = nb * BN + (kCta == 2 ? static_cast<int>(rank) * 128 : 0);
+      // double-width tile: whether its second 256 columns hold any of D (else
+      // that half is neither loaded nor multiplied)
+      const bool half1 = kDbl && nb * BN + 256 < p.N;
+      const uint32_t tx_bytes = kDbl ? (half1 ? STAGE_BYTES : A_BYTES + B_HALF_BYTES) : STAGE_BYTES;
       bool ok = true;
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!wait_bar<kCta>(empty_bar(stage), phase ^ 1u, abort_flag, kSiteProducerEmpty,
@@ -351,7 +375,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
         const uint32_t fb = full_bar(stage);
         if (leader) {
-          mbar_arrive_expect_tx(fb, kCta * STAGE_BYTES);
+          mbar_arrive_expect_tx(fb, kCta * tx_bytes);
           armed_mask |= 1u << stage;
           armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
         }
@@ -364,6 +388,10 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           else      tma_load_2d_pair(a_dst, &tmap_a, fb_leader, k0, a_row);
           if (kBMN) tma_load_2d_pair(b_dst, &tmap_b, fb_leader, b_row, k0);
           else      tma_load_2d_pair(b_dst, &tmap_b, fb_leader, k0, b_row);
+          if (half1) {
+            if (kBMN) tma_load_2d_pair(b_dst + B_HALF_BYTES, &tmap_b, fb_leader, b_row + 256, k0);
+            else      tma_load_2d_pair(b_dst + B_HALF_BYTES, &tmap_b, fb_leader, k0, b_row + 256);
+          }
         } else {
           if (kAMN) tma_load_2d(a_dst, &tmap_a, fb, a_row, k0);
           else      tma_load_2d(a_dst, &tmap_a, fb, k0, a_row);
@@ -396,15 +424,61 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       const int t = u / p.splits;
       const int kb0 = (u - t * p.splits) * p.kb_per_split;
       const int kb1 = min(kb0 + p.kb_per_split, p.num_k_blocks);
-      const int acc = local & 1;
-      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      const int acc = kDbl ? 0 : (local & 1);
+      const uint32_t use = static_cast<uint32_t>(kDbl ? local : (local >> 1));
+      int mb_, nb_;
+      tile_coords(t, p, mb_, nb_);
+      const bool half1 = kDbl && nb_ * BN + 256 < p.N;
       if (!wait_bar<kCta>(tempty_bar(acc), (use & 1u) ^ 1u, abort_flag, kSiteMmaTmemEmpty,
                           p.wait_limit_ns))
         break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
       bool ok = true;
-      for (int kb = kb0; kb < kb1; ++kb) {
+      // Double-width tile: the epilogue frees columns 0..255 of the single
+      // accumulator before 256..511.  The first `defer` stages of a tile are
+      // multiplied into the first half only, while the second half drains;
+      // their second-half MMAs follow once it is free, and only then are
+      // those stages released (at most STAGES are held, all of which the
+      // producer can fill).  The rest run both halves stage by stage.
+      int defer = 0;
+      if (kDbl) {
+        defer = min(STAGES, kb1 - kb0);
+        int st = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < defer; ++i) {
+          if (!wait_bar<kCta>(full_bar(st), ph, abort_flag, kSiteMmaFull, p.wait_limit_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + st * A_BYTES);
+          const uint32_t b_base = smem_u32(sB + st * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UK; ++k)
+            mma_f8f6f4_pair(d_tmem, operand_desc<kAMN>(a_base, k), operand_desc<kBMN>(b_base, k),
+                            p.idesc, (i != 0 || k != 0) ? 1u : 0u);
+          if (++st == STAGES) { st = 0; ph ^= 1u; }
+        }
+        if (ok && !wait_bar<kCta>(tempty_bar(1), (use & 1u) ^ 1u, abort_flag, kSiteMmaTmemEmpty,
+                                  p.wait_limit_ns))
+          ok = false;
+        if (!ok) break;
+        tc_fence_after();
+        for (int i = 0; i < defer; ++i) {
+          if (half1) {
+            const uint32_t a_base = smem_u32(sA + stage * A_BYTES);
+            const uint32_t b_base = smem_u32(sB + stage * B_BYTES) + B_HALF_BYTES;
+#pragma unroll
+            for (int k = 0; k < BK / UK; ++k)
+              mma_f8f6f4_pair(d_tmem + 256u, operand_desc<kAMN>(a_base, k),
+                              operand_desc<kBMN>(b_base, k), p.idesc, (i != 0 || k != 0) ? 1u : 0u);
+          }
+          mma_commit_pair_mc(empty_bar(stage), 0x3);   // both halves have read the stage
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      for (int kb = kb0 + defer; kb < kb1; ++kb) {
         if (!wait_bar<kCta>(full_bar(stage), phase, abort_flag, kSiteMmaFull, p.wait_limit_ns)) {
           ok = false;
           break;
@@ -419,6 +493,12 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           const uint32_t accum = (kb != kb0 || k != 0) ? 1u : 0u;
           if (kCta == 2) mma_f8f6f4_pair(d_tmem, ad, bd, p.idesc, accum);
           else           mma_f8f6f4(d_tmem, ad, bd, p.idesc, accum);
+        }
+        if (kDbl && half1) {
+#pragma unroll
+          for (int k = 0; k < BK / UK; ++k)
+            mma_f8f6f4_pair(d_tmem + 256u, operand_desc<kAMN>(a_base, k),
+                            operand_desc<kBMN>(b_base + B_HALF_BYTES, k), p.idesc, 1u);
         }
         // frees the stage (in both CTAs) once these MMAs have read it
         if (kCta == 2) mma_commit_pair_mc(empty_bar(stage), 0x3);
@@ -445,8 +525,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     for (int u = unit; u < p.num_work; u += num_units, ++local) {
       const int t = u / p.splits;
       const int split = u - t * p.splits;
-      const int acc = local & 1;
-      const uint32_t use = static_cast<uint32_t>(local >> 1);
+      const int acc = kDbl ? 0 : (local & 1);
+      const uint32_t use = static_cast<uint32_t>(kDbl ? local : (local >> 1));
       int ok = 1;
       if (lane == 0)
         ok = wait_bar<kCta>(tfull_bar(acc), use & 1u, abort_flag, kSiteEpilogueTmemFull,
@@ -458,11 +538,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       tile_coords(t, p, mb, nb);
       const int64_t row = static_cast<int64_t>(mb) * C::BM + row_in_tile;
       const bool row_ok = row < p.M;
-      if (kCta == 1 && p.splits > 1) {
-        // ---- split K: store this range's raw fp32 partial, free the
-        // accumulator, and let the last range to finish these 32 rows of the
-        // tile (one counter per tile and warp quarter, so the four epilogue
-        // warps never wait on each other) add the partials and store them
+      if (!kDbl && p.splits > 1) {
+        // ---- split K: store this range's raw fp32 partial and free the
+        // accumulator; splitk_reduce_kernel sums the ranges afterwards
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           const int col0 = nb * BN + c * 32;
@@ -483,55 +561,42 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           }
         }
         tc_fence_before();
-        __threadfence();                          // partial visible before the count
         __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar(acc));
-        uint32_t prev = 0;
-        if (lane == 0) prev = atomicAdd(&p.counters[t * 4 + quarter], 1u);
-        prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-        if (prev != static_cast<uint32_t>(p.splits - 1)) continue;
-        __threadfence();                          // all partials visible to this warp
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          const int col0 = nb * BN + c * 32;
-          if (col0 >= p.N) break;
-          if (!row_ok) continue;
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0.0f;
-          for (int sp = 0; sp < p.splits; ++sp) {     // fixed order: deterministic sum
-            const float4* src = reinterpret_cast<const float4*>(
-                p.ws + (static_cast<int64_t>(sp) * p.M + row) * p.N + col0);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (col0 + 4 * j < p.N) {
-                const float4 q = __ldcg(src + j);
-                v[4 * j] += q.x; v[4 * j + 1] += q.y; v[4 * j + 2] += q.z; v[4 * j + 3] += q.w;
-              }
-            }
-          }
-          uint32_t r[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(v[j]);
-          store_row_chunk<kOutF32, kAmax>(p, row, col0, r, sc, dmax);
+        if (lane == 0) {
+          if (kCta == 2) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+          else           mbar_arrive(tempty_bar(acc));
         }
         continue;
       }
+      constexpr int kChunks = BN / 32 / kHalves;  // 32-column chunks per half
+      static_assert(kChunks % 2 == 0, "chunks are drained in pairs");
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int col0 = nb * BN + c * 32;
-        if (col0 >= p.N) break;                   // warp-uniform
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                               static_cast<uint32_t>(acc * BN + c * 32), r);
-        tmem_ld_wait();
-        if (row_ok) store_row_chunk<kOutF32, kAmax>(p, row, col0, r, sc, dmax);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (kCta == 2) mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));  // leader's barrier
-        else           mbar_arrive(tempty_bar(acc));
+      for (int h = 0; h < kHalves; ++h) {
+        // two 32-column loads in flight per wait (kChunks is even)
+#pragma unroll 1
+        for (int c = h * kChunks; c < (h + 1) * kChunks; c += 2) {
+          const int col0 = nb * BN + c * 32;
+          if (col0 >= p.N) break;                 // warp-uniform
+          const bool two = col0 + 32 < p.N;       // warp-uniform
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                 static_cast<uint32_t>(acc * BN + c * 32);
+          uint32_t r0[32], r1[32];
+          tmem_ld_32x32b_x32(taddr, r0);
+          if (two) tmem_ld_32x32b_x32(taddr + 32u, r1);
+          tmem_ld_wait();
+          if (row_ok) {
+            store_row_chunk<kOutF32, kAmax>(p, row, col0, r0, sc, dmax);
+            if (two) store_row_chunk<kOutF32, kAmax>(p, row, col0 + 32, r1, sc, dmax);
+          }
+        }
+        // these columns are free for the next tile's MMAs
+        tc_fence_before();
+        __syncwarp();
+        const uint32_t tb = tempty_bar(kDbl ? h : acc);
+        if (lane == 0) {
+          if (kCta == 2) mbar_arrive_cluster(mapa_shared(tb, 0));  // leader's barrier
+          else           mbar_arrive(tb);
+        }
       }
     }
     if (kAmax) {
@@ -566,6 +631,63 @@ __global__ void selftest_wait_kernel(uint64_t limit_ns) {
     mbar_init(smem_u32(&bar), 1);
     fence_mbarrier_init();
     mbar_wait_bounded(smem_u32(&bar), 0, &abort_flag, kSiteSelfTest, limit_ns);
+  }
+}
+
+// Split-K epilogue: D = (sum over ranges of ws[range]) * 2^-(bias_a+bias_b),
+// one rounding to the output type (fp32 sums in range order: the result does
+// not depend on which unit finished first).  A separate launch rather than
+// "the last unit of a tile adds the partials": that left one CTA per tile
+// reading all of the tile's partials with a few loads in flight per thread,
+// while here every SM streams them, all ranges' loads of a 4-column group in
+// flight together.  N % 4 == 0, so a 4-column group never crosses a row.
+constexpr int kReduceThreads = 256;
+constexpr int kReduceUnroll = 8;     // ranges whose loads are issued together
+
+template <bool kOutF32, bool kAmax>
+__global__ void __launch_bounds__(kReduceThreads)
+splitk_reduce_kernel(const float4* __restrict__ ws, int splits, int64_t n4,
+                     const int32_t* bias_a, const int32_t* bias_b, void* d, uint32_t* amax_out) {
+  const Pow2Scale sc = make_pow2_scale(-(*bias_a + *bias_b));
+  uint32_t dmax = 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += stride) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < splits; s0 += kReduceUnroll) {
+      float4 v[kReduceUnroll];
+#pragma unroll
+      for (int u = 0; u < kReduceUnroll; ++u)
+        if (s0 + u < splits) v[u] = __ldcs(ws + static_cast<int64_t>(s0 + u) * n4 + i);
+#pragma unroll
+      for (int u = 0; u < kReduceUnroll; ++u) {
+        if (s0 + u < splits) {
+          acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+        }
+      }
+    }
+    const float x = apply_pow2(acc.x, sc), y = apply_pow2(acc.y, sc);
+    const float z = apply_pow2(acc.z, sc), w = apply_pow2(acc.w, sc);
+    if (kOutF32) {
+      reinterpret_cast<float4*>(d)[i] = make_float4(x, y, z, w);
+      if (kAmax)
+        dmax = max(dmax, max(max(__float_as_uint(x) & 0x7FFFFFFFu, __float_as_uint(y) & 0x7FFFFFFFu),
+                             max(__float_as_uint(z) & 0x7FFFFFFFu, __float_as_uint(w) & 0x7FFFFFFFu)));
+    } else {
+      uint2 o;
+      o.x = pack_bf16x2(x, y);
+      o.y = pack_bf16x2(z, w);
+      reinterpret_cast<uint2*>(d)[i] = o;
+      if (kAmax) {
+        dmax = __vmaxu2(dmax, o.x & 0x7FFF7FFFu);
+        dmax = __vmaxu2(dmax, o.y & 0x7FFF7FFFu);
+      }
+    }
+  }
+  if (kAmax) {
+    uint32_t bits = kOutF32 ? dmax : (max(dmax & 0xFFFFu, dmax >> 16) << 16);
+    bits = __reduce_max_sync(0xFFFFFFFFu, bits);
+    if ((threadIdx.x & 31) == 0 && bits != 0u) atomicMax(amax_out, bits);
   }
 }
 
@@ -626,13 +748,12 @@ int sm_count() {
 // that sweep one whole operand (M fastest or N fastest) by 1-5 %, except
 // where both operands are large (K = 28672: both > 128 MB), where 8 won by
 // 1-2 %; an evict-last hint on either operand only slowed it down.
-// Split-K workspace: fp32 partials [splits][M][N] (256-byte aligned), then
-// one uint32 counter per tile and epilogue warp (4 per tile).
+// Split-K workspace: fp32 partials [splits][M][N] (256-byte aligned).
 size_t splitk_partials_bytes(int splits, int64_t M, int64_t N) {
   return ((static_cast<size_t>(splits) * M * N * sizeof(float)) + 255) & ~size_t(255);
 }
-size_t splitk_workspace_bytes(int splits, int64_t M, int64_t N, int num_tiles) {
-  return splitk_partials_bytes(splits, M, N) + 4 * sizeof(uint32_t) * static_cast<size_t>(num_tiles);
+size_t splitk_workspace_bytes(int splits, int64_t M, int64_t N) {
+  return splitk_partials_bytes(splits, M, N);
 }
 
 int pick_group_n(uint64_t a_bytes, uint64_t b_bytes) {
@@ -660,6 +781,33 @@ int plan_splits(int64_t M, int num_tiles, int num_k_blocks, int* kb_per_split) {
   return (num_k_blocks + per - 1) / per;     // no empty range
 }
 
+// Split K for CTA-pair tiles (M > 128) when the 256 x 256 tiles cannot fill
+// half of the pairs: small outputs with a long K, e.g. the weight gradients
+// of small layers (GPT-111M: a 768 x 768 dW over 8192 tokens is 9 tiles for 74
+// pairs).  At least 8 k-blocks per range.
+int plan_pair_splits(int num_tiles, int num_k_blocks, int num_pairs, int* kb_per_split) {
+  int splits = 1;
+  if (2 * num_tiles <= num_pairs) {
+    splits = num_pairs / num_tiles;
+    splits = splits < num_k_blocks / 8 ? splits : num_k_blocks / 8;
+    splits = splits < 16 ? splits : 16;
+    if (splits < 1) splits = 1;
+  }
+  int per = (num_k_blocks + splits - 1) / splits;
+  *kb_per_split = per;
+  return (num_k_blocks + per - 1) / per;
+}
+
+// Pairs the pair kernels may run at once on this device: the occupancy query
+// made at their first launch, or one pair per two SMs before that.
+int g_pair_units[64];
+int pair_units() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  return g_pair_units[dev] > 0 ? g_pair_units[dev] : sm_count() / 2;
+}
+
 template <int kTile, bool kAMN, bool kBMN, bool kOutF32, bool kAmax>
 int launch_t(const GemmArgs& g, cudaStream_t s) {
   constexpr int kCta = Cfg<kTile>::CTAS;
@@ -669,7 +817,7 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
   // TMA boxes: 128 x 128 bytes for A (this CTA's rows); for a K-major B, the
   // CTA's B rows (256, 128 or 64) x 128 bytes; for an MN-major B, 128 MN
   // columns x 128 K rows (the single-CTA tile loads two of them).
-  const uint32_t b_box_rows = kBMN ? 128 : Cfg<kTile>::B_ROWS;
+  const uint32_t b_box_rows = (kBMN || kTile == kTileDouble) ? 128 : Cfg<kTile>::B_ROWS;
   CUtensorMap ta, tb;
   const uint64_t M = g.M, N = g.N, K = g.K;
   const bool ok_a = kAMN ? encode_2d(&ta, g.a, M, K, 128, BK) : encode_2d(&ta, g.a, K, M, BK, 128);
@@ -686,23 +834,20 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
   p.num_k_blocks = (p.K + BK - 1) / BK;
   p.num_tiles = p.num_m_blocks * p.num_n_blocks;
   p.group_n = pick_group_n(M * K, N * K);
+  if (kTile == kTileDouble) p.group_n /= 2;   // the same columns in half as many tiles
   p.splits = 1;
   p.kb_per_split = p.num_k_blocks;
   p.ws = nullptr;
-  p.counters = nullptr;
-  if (g.workspace != nullptr && kCta == 1) {
+  if (g.workspace != nullptr && kTile != kTileDouble) {
     int per = 0;
-    const int sp = plan_splits(g.M, p.num_tiles, p.num_k_blocks, &per);
+    const int sp = kCta == 1 ? plan_splits(g.M, p.num_tiles, p.num_k_blocks, &per)
+                             : plan_pair_splits(p.num_tiles, p.num_k_blocks, pair_units(), &per);
     if (sp > 1) {
-      const size_t need = splitk_workspace_bytes(sp, g.M, g.N, p.num_tiles);
+      const size_t need = splitk_workspace_bytes(sp, g.M, g.N);
       if (need > g.workspace_bytes) return FP8_ERR_INVALID_ARGUMENT;
       p.splits = sp;
       p.kb_per_split = per;
       p.ws = static_cast<float*>(g.workspace);
-      p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(g.workspace) +
-                                               splitk_partials_bytes(sp, g.M, g.N));
-      if (cudaMemsetAsync(p.counters, 0, 4 * sizeof(uint32_t) * p.num_tiles, s) != cudaSuccess)
-        return FP8_ERR_CUDA;
     }
   }
   p.num_work = p.num_tiles * p.splits;
@@ -711,7 +856,7 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
             | (static_cast<uint32_t>(g.b_fmt) << 10)      // B: 0 E4M3, 1 E5M2
             | (static_cast<uint32_t>(kAMN) << 15)         // A major: 0 K, 1 MN
             | (static_cast<uint32_t>(kBMN) << 16)         // B major
-            | (static_cast<uint32_t>(BN >> 3) << 17)      // N / 8
+            | (static_cast<uint32_t>(Cfg<kTile>::MMA_N >> 3) << 17)   // N / 8 of one MMA
             | (static_cast<uint32_t>(BM >> 4) << 24);     // M / 16 (256 for a pair)
   p.bias_a = g.bias_a;
   p.bias_b = g.bias_b;
@@ -751,12 +896,22 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
         clusters = sm_count() / 2;
       }
       units = clusters;
+      if (g_pair_units[dev] == 0 || clusters < g_pair_units[dev]) g_pair_units[dev] = clusters;
     }
     max_units[dev] = units;
   }
   const int units = p.num_work < max_units[dev] ? p.num_work : max_units[dev];
   cfg.gridDim = dim3(static_cast<unsigned>(units * kCta), 1, 1);
   if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return FP8_ERR_CUDA;
+  if (p.splits > 1) {
+    const int64_t n4 = static_cast<int64_t>(g.M) * g.N / 4;
+    int64_t blocks = (n4 + kReduceThreads - 1) / kReduceThreads;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+    if (blocks > cap) blocks = cap;
+    splitk_reduce_kernel<kOutF32, kAmax><<<static_cast<unsigned>(blocks), kReduceThreads, 0, s>>>(
+        reinterpret_cast<const float4*>(p.ws), p.splits, n4, g.bias_a, g.bias_b, g.d,
+        p.amax_out);
+  }
   return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
@@ -766,20 +921,47 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
 // leave more than half of the SMs idle and the narrow ones still fit in one
 // wave (measured on the Llama-2-70B projections at T <= 128: a second, mostly
 // empty wave of narrow tiles costs more than the idle SMs of the wide ones).
+constexpr double kDoubleGain = 1.05;
+
 bool few_wide_tiles(int64_t M, int64_t N) {
   const int64_t wide = ((M + 127) / 128) * ((N + 255) / 256);
   return M <= 128 && 2 * wide <= sm_count();
 }
 
-template <bool kAMN, bool kBMN, bool kOutF32, bool kAmax = false>
-int launch_pick(const GemmArgs& g, cudaStream_t s) {
+// 256 x 512 pair tiles where they fill the GPU about as evenly as 256 x 256
+// ones: the fraction of pair-slots busy over the waves of each tile shape,
+// the wide one credited with its lower L2 traffic per FLOP.
+bool use_double(const GemmArgs& g) {
+  if (g.M <= 128 || g.N <= 256) return false;
+  const int64_t pairs = pair_units();
+  const int64_t mb = (g.M + 255) / 256;
+  const int64_t t256 = mb * ((g.N + 255) / 256);
+  const int64_t t512 = mb * ((g.N + 511) / 512);
+  const double e256 = static_cast<double>(t256) / (((t256 + pairs - 1) / pairs) * pairs);
+  const double e512 = static_cast<double>(t512) / (((t512 + pairs - 1) / pairs) * pairs);
+  return e512 * kDoubleGain >= e256;
+}
+
+int choose_tile(const GemmArgs& g) {
+  if (g.workspace == nullptr && use_double(g)) return kTileDouble;
   if (g.M <= 128) {
     const int64_t narrow = (g.N + 63) / 64;
-    if (!kBMN && g.workspace == nullptr && few_wide_tiles(g.M, g.N) && narrow <= sm_count())
-      return launch_t<kTileNarrow, kAMN, false, kOutF32, kAmax>(g, s);
-    return launch_t<kTileSingle, kAMN, kBMN, kOutF32, kAmax>(g, s);
+    if (!g.b_mn_major && g.workspace == nullptr && few_wide_tiles(g.M, g.N) &&
+        narrow <= sm_count())
+      return kTileNarrow;
+    return kTileSingle;
   }
-  return launch_t<kTilePair, kAMN, kBMN, kOutF32, kAmax>(g, s);
+  return kTilePair;
+}
+
+template <bool kAMN, bool kBMN, bool kOutF32, bool kAmax = false>
+int launch_pick(const GemmArgs& g, cudaStream_t s) {
+  switch (choose_tile(g)) {
+    case kTileDouble: return launch_t<kTileDouble, kAMN, kBMN, kOutF32, kAmax>(g, s);
+    case kTileNarrow: return launch_t<kTileNarrow, kAMN, false, kOutF32, kAmax>(g, s);
+    case kTileSingle: return launch_t<kTileSingle, kAMN, kBMN, kOutF32, kAmax>(g, s);
+    default:          return launch_t<kTilePair, kAMN, kBMN, kOutF32, kAmax>(g, s);
+  }
 }
 
 }  // namespace
@@ -810,13 +992,39 @@ int launch_gemm(const GemmArgs& g, cudaStream_t s) {
   }
 }
 
+void gemm_plan(const GemmArgs& g, GemmPlan* plan) {
+  GemmArgs h = g;
+  const size_t need = gemm_workspace_bytes(g);
+  if (g.workspace == nullptr || need == 0) h.workspace = nullptr;
+  const int kind = choose_tile(h);
+  int bm = 256, bn = 256, ctas = 2;
+  if (kind == kTileDouble) bn = 512;
+  if (kind == kTileSingle || kind == kTileNarrow) { bm = 128; ctas = 1; }
+  if (kind == kTileNarrow) bn = 64;
+  const int nkb = static_cast<int>((g.K + BK - 1) / BK);
+  const int tiles = static_cast<int>(((g.M + bm - 1) / bm) * ((g.N + bn - 1) / bn));
+  int splits = 1, per = 0;
+  if (h.workspace != nullptr)
+    splits = ctas == 1 ? plan_splits(g.M, tiles, nkb, &per)
+                       : plan_pair_splits(tiles, nkb, pair_units(), &per);
+  plan->tile_m = bm;
+  plan->tile_n = bn;
+  plan->ctas_per_tile = ctas;
+  plan->k_splits = splits;
+}
+
 size_t gemm_workspace_bytes(const GemmArgs& g) {
-  if (!few_wide_tiles(g.M, g.N)) return 0;
-  const int tiles = static_cast<int>(((g.M + 127) / 128) * ((g.N + 255) / 256));
   const int nkb = static_cast<int>((g.K + BK - 1) / BK);
   int per = 0;
+  if (g.M > 128) {
+    const int tiles = static_cast<int>(((g.M + 255) / 256) * ((g.N + 255) / 256));
+    const int sp = plan_pair_splits(tiles, nkb, pair_units(), &per);
+    return sp > 1 ? splitk_workspace_bytes(sp, g.M, g.N) : 0;
+  }
+  if (!few_wide_tiles(g.M, g.N)) return 0;
+  const int tiles = static_cast<int>(((g.M + 127) / 128) * ((g.N + 255) / 256));
   const int sp = plan_splits(g.M, tiles, nkb, &per);
-  return sp > 1 ? splitk_workspace_bytes(sp, g.M, g.N, tiles) : 0;
+  return sp > 1 ? splitk_workspace_bytes(sp, g.M, g.N) : 0;
 }
 
 // ----------------------------------------------------------------------------
@@ -845,12 +1053,13 @@ int launch_gemm_noalloc(GemmArgs g, cudaStream_t s) {
       return FP8_ERR_CUDA;
     scratch_addr[dev] = ptr;
   }
-  const size_t need = gemm_workspace_bytes(g);
-  if (need > kNoAllocScratchBytes) return FP8_ERR_UNSUPPORTED;
+  size_t need = gemm_workspace_bytes(g);
+  if (need > kNoAllocScratchBytes) {
+    if (g.M <= 128) return FP8_ERR_UNSUPPORTED;
+    need = 0;     // CTA-pair tiles: split only when the partials fit, else run unsplit
+  }
   if (need > 0) {
-    // the split counters the kernel needs at zero are cleared by launch_gemm
-    // (a memset inside the array) before every launch; the fp32 partials are
-    // always written before they are read
+    // every fp32 partial is written by the GEMM before the reduction reads it
     g.workspace = scratch_addr[dev];
     g.workspace_bytes = kNoAllocScratchBytes;
   }

@@ -41,6 +41,14 @@ int launch_gemm(const GemmArgs& g, cudaStream_t s);
 // one (0: the problem is never split).  a/b/d pointers are not read.
 size_t gemm_workspace_bytes(const GemmArgs& g);
 
+// The launch launch_gemm makes for this problem: tile shape, CTAs per tile
+// and K splits.  `g.workspace` non-null means the caller supplies
+// gemm_workspace_bytes(g) bytes.  a/b/d pointers are not read.
+struct GemmPlan {
+  int tile_m, tile_n, ctas_per_tile, k_splits;
+};
+void gemm_plan(const GemmArgs& g, GemmPlan* plan);
+
 // launch_gemm with the split-K scratch taken from a static device array
 // instead of a caller workspace (FP8_ERR_UNSUPPORTED beyond its 16 MiB).
 int launch_gemm_noalloc(GemmArgs g, cudaStream_t s);

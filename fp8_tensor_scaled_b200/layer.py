@@ -25,7 +25,8 @@ Every operation is one call of the C library (see ``__init__``).
 import torch
 
 from . import (E4M3, E5M2, fp8_cast_scaled, fp8_linear_bwd_dgrad, fp8_linear_bwd_wgrad,
-               fp8_linear_fwd, fp8_quantize)
+               fp8_linear_bwd_wgrad_workspace_size, fp8_linear_bwd_wgrad_ws, fp8_linear_fwd,
+               fp8_quantize)
 
 
 class Fp8AmaxLinear:
@@ -52,10 +53,15 @@ class Fp8AmaxLinear:
                 raise ValueError("fixed_bias is (bias_x, bias_w, bias_dy)")
             self.bias.copy_(torch.tensor(self.fixed, dtype=torch.int32))
         self.y = torch.empty((self.T, self.outf), dtype=out_dtype, device=dev)
+        self.wgrad_ws = None
         if backward:
             self.dy8 = torch.empty((self.T, self.outf), **u8)
             self.dx = torch.empty((self.T, self.inf), dtype=out_dtype, device=dev)
             self.dw = torch.empty((self.outf, self.inf), dtype=out_dtype, device=dev)
+            # a small dW over many tokens splits K across more CTA pairs
+            ws = fp8_linear_bwd_wgrad_workspace_size(self.T, self.inf, self.outf)
+            if ws > 0:
+                self.wgrad_ws = torch.empty(ws, **u8)
 
     def quantize(self, x, w, dy=None):
         """Cast X, W (E4M3) and dY (E5M2).  On refresh steps amax -> bias ->
@@ -71,12 +77,26 @@ class Fp8AmaxLinear:
             else:
                 fp8_cast_scaled(t, self.bias[i:i + 1], fmt, out=out)
 
-    def gemms(self):
+    def gemms(self, pass_done=None):
+        """The three GEMMs on the current stream.  `pass_done` (optional): one
+        CUDA event per pass (fwd, dgrad, wgrad), each recorded as soon as that
+        pass's output is complete, so a consumer can take Y before dX and dW
+        are done."""
         bx, bw, bdy = self.bias[0:1], self.bias[1:2], self.bias[2:3]
         fp8_linear_fwd(self.x8, E4M3, bx, self.w8, E4M3, bw, out=self.y)
+        if pass_done is not None:
+            pass_done[0].record()
         if self.backward:
             fp8_linear_bwd_dgrad(self.dy8, E5M2, bdy, self.w8, E4M3, bw, out=self.dx)
-            fp8_linear_bwd_wgrad(self.dy8, E5M2, bdy, self.x8, E4M3, bx, out=self.dw)
+            if pass_done is not None:
+                pass_done[1].record()
+            if self.wgrad_ws is not None:
+                fp8_linear_bwd_wgrad_ws(self.dy8, E5M2, bdy, self.x8, E4M3, bx, out=self.dw,
+                                        workspace=self.wgrad_ws)
+            else:
+                fp8_linear_bwd_wgrad(self.dy8, E5M2, bdy, self.x8, E4M3, bx, out=self.dw)
+            if pass_done is not None:
+                pass_done[2].record()
 
     def step(self, x, w, dy=None):
         self.quantize(x, w, dy)
@@ -106,7 +126,7 @@ class Fp8AmaxStep:
         host call: no per-kernel launch cost, which matters for small layers.
     ``step_from_host(h_in, d_in, h_out)``  the same step from pinned host tensors:
         copies in on one copy stream, copies of each linear's Y, dX, dW out on
-        another as soon as its GEMMs finish, so transfers in both directions
+        another as soon as the pass that writes it finishes, so transfers in both directions
         overlap each other and the compute.  Returns when the caller's stream
         has been ordered after the last copy out.
     """
@@ -123,6 +143,7 @@ class Fp8AmaxStep:
         self.q_done = [torch.cuda.Event() for _ in range(n)]
         self.in_done = [torch.cuda.Event() for _ in range(n)]
         self.g_done = [torch.cuda.Event() for _ in range(n)]
+        self.p_done = [[torch.cuda.Event() for _ in range(3)] for _ in range(n)]
         self.out_done = torch.cuda.Event()
 
     def flops(self):
@@ -156,7 +177,7 @@ class Fp8AmaxStep:
             main.wait_event(self.q_done[i])
             if timing is not None:
                 timing["g"][i][0].record(main)
-            self.linears[i].gemms()
+            self.linears[i].gemms(self.p_done[i])
             if timing is not None:
                 timing["g"][i][1].record(main)
             self.g_done[i].record(main)
@@ -195,9 +216,11 @@ class Fp8AmaxStep:
                 self.in_done[i].record(self.h2d)
         self.step(device_inputs, in_events=self.in_done)
         with torch.cuda.stream(self.d2h):
+            # each output leaves as soon as its own pass is done: the copy of
+            # Y overlaps dgrad and wgrad, so the last copy out starts earlier
             for i, (lin, hs) in enumerate(zip(self.linears, host_outputs)):
-                self.d2h.wait_event(self.g_done[i])
-                for h, d in zip(hs, (lin.y, lin.dx, lin.dw)):
+                for k, (h, d) in enumerate(zip(hs, (lin.y, lin.dx, lin.dw))):
+                    self.d2h.wait_event(self.p_done[i][k])
                     h.copy_(d, non_blocking=True)
             self.out_done.record(self.d2h)
         main.wait_event(self.out_done)

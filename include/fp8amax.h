@@ -49,6 +49,7 @@ typedef enum {
 
 typedef enum { FP8_E4M3 = 0, FP8_E5M2 = 1 } fp8_format_t;     /* FP8_E4 / FP8_E5 of the page */
 typedef enum { FP8_DTYPE_BF16 = 0, FP8_DTYPE_FP32 = 1 } fp8_dtype_t;
+typedef enum { FP8_PASS_FWD = 0, FP8_PASS_DGRAD = 1, FP8_PASS_WGRAD = 2 } fp8_pass_t;
 
 /*
  * Step 1 — per-tensor amax ("Proposed method": maximum absolute value of the
@@ -151,12 +152,13 @@ fp8_status_t fp8_linear_bwd_dgrad_amax(const uint8_t *dy8, fp8_format_t fdy,
                                        void *stream);
 
 /*
- * fp8_linear_fwd for few tokens (T <= 64, e.g. decode-sized inference calls),
- * where the GEMM streams the weights and one tile per 128 x 256 block of Y
- * leaves SMs idle: with a caller-provided workspace a long K dimension is
- * split across more CTAs, each writing an fp32 partial to the workspace, and
- * the last CTA of each tile adds the partials in a fixed order (deterministic)
- * before the unscale and the single rounding.  Results equal fp8_linear_fwd's
+ * fp8_linear_fwd with a split-K workspace.  For few tokens (T <= 64, e.g.
+ * decode-sized inference calls) the GEMM streams the weights and one tile per
+ * 128 x 256 block of Y leaves SMs idle; for more tokens, outputs with too few
+ * 256 x 256 tiles to fill half the GPU.  With a caller-provided workspace a
+ * long K dimension is split across more CTAs, each writing an fp32 partial to
+ * the workspace; a second kernel on the same stream adds the partials in a
+ * fixed order (deterministic) before the unscale and the single rounding.  Results equal fp8_linear_fwd's
  * within the GEMM tolerance (the fp32 summation order differs); shapes that do
  * not split run exactly as fp8_linear_fwd.
  *   fp8_linear_fwd_workspace_size(T, in, out) returns the bytes needed (0
@@ -175,6 +177,48 @@ fp8_status_t fp8_linear_fwd_ws(const uint8_t *x8, fp8_format_t fx, const int32_t
                                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * fp8_linear_bwd_wgrad with a split-K workspace, for weight gradients whose
+ * output [out, in] has too few 256 x 256 tiles to fill the GPU while K = T is
+ * long (small layers over many tokens: a 768 x 768 dW over 8192 tokens is 9
+ * tiles).  K is split across more CTA pairs, each writing an fp32 partial;
+ * a second kernel adds them in a fixed order (deterministic) and runs the
+ * epilogue.  Results equal fp8_linear_bwd_wgrad's within the GEMM
+ * tolerance; problems that do not split run exactly as fp8_linear_bwd_wgrad.
+ * fp8_linear_bwd_wgrad_workspace_size returns the bytes needed (0: no split).
+ * Workspace rules as for fp8_linear_fwd_ws.
+ */
+size_t fp8_linear_bwd_wgrad_workspace_size(int64_t T, int64_t in, int64_t out);
+
+fp8_status_t fp8_linear_bwd_wgrad_ws(const uint8_t *dy8, fp8_format_t fdy, const int32_t *bias_dy,
+                                     const uint8_t *x8, fp8_format_t fx, const int32_t *bias_x,
+                                     int64_t T, int64_t in, int64_t out, void *dw,
+                                     fp8_dtype_t dw_dtype, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
+/*
+ * The launch plan of one GEMM pass on the current device, for performance
+ * work and for tests that must know which kernel shape ran.  The paper has no
+ * counterpart.  Nothing is launched and no data pointer is involved.
+ *   pass            FP8_PASS_FWD (Y = X.W^T, M = T, N = out, K = in),
+ *                   FP8_PASS_DGRAD (dX = dY.W, M = T, N = in, K = out) or
+ *                   FP8_PASS_WGRAD (dW = dY^T.X, M = out, N = in, K = T).
+ *   with_workspace  nonzero: the plan of fp8_linear_fwd_ws / _bwd_wgrad_ws
+ *                   given the workspace their size query asks for (ignored
+ *                   for DGRAD, which has no such entry point).
+ *   plan            out: output tile rows and columns, CTAs that compute one
+ *                   tile (1, or 2 for a CTA pair) and the number of ranges
+ *                   K is split into (1: not split).
+ * Returns FP8_ERR_INVALID_ARGUMENT for a null plan, a negative size or an
+ * unknown pass, FP8_ERR_NO_DEVICE without an sm_100 device.
+ */
+typedef struct {
+    int32_t tile_m, tile_n, ctas_per_tile, k_splits;
+} fp8_gemm_plan_t;
+
+fp8_status_t fp8_linear_plan(fp8_pass_t pass, int64_t T, int64_t in, int64_t out,
+                             int with_workspace, fp8_gemm_plan_t *plan);
+
+/*
  * fp8_linear_fwd_ws for callers that cannot allocate device memory when they
  * run a forward (an allocator that must not be entered there, a fixed memory
  * pool, a serving loop that forbids allocation, a C program with no device
@@ -186,9 +230,11 @@ fp8_status_t fp8_linear_fwd_ws(const uint8_t *x8, fp8_format_t fx, const int32_t
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
  *   - Nothing is allocated, by this call or below it.
- *   - A problem whose split-K scratch would exceed 16 MiB (only possible for
- *     T <= 64 with very wide outputs) returns FP8_ERR_UNSUPPORTED; problems
- *     that do not split use no scratch at all.
+ *   - A problem with T <= 128 whose split-K scratch would exceed 16 MiB
+ *     (only possible for T <= 64 with very wide outputs) returns
+ *     FP8_ERR_UNSUPPORTED; for T > 128 a split whose partials would not fit
+ *     is not made and the forward runs unsplit; problems that do not split
+ *     use no scratch at all.
  *   - All calls share the one array and it keeps the last call's contents:
  *     calls that overlap on the GPU (different streams, no ordering between
  *     them) race on it and must be serialised by the caller.

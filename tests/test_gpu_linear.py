@@ -307,6 +307,8 @@ def test_split_k_few_tokens(T, out_dtype):
     qw, bw, rqw, rbw, fw = Q["w"]
     need = fp8.fp8_linear_fwd_workspace_size(T, In, Out)
     assert (need > 0) == (T <= 64)
+    plan = fp8.fp8_linear_plan(fp8.FWD, T, In, Out, with_workspace=True)
+    assert (plan["k_splits"] > 1) == (T <= 64) and plan["tile_m"] == 128, plan
     y1 = fp8.fp8_linear_fwd_ws(qx, fx, bx, qw, fw, bw, out_dtype=out_dtype)
     y2 = fp8.fp8_linear_fwd_ws(qx, fx, bx, qw, fw, bw, out_dtype=out_dtype)
     torch.cuda.synchronize()
@@ -336,6 +338,16 @@ def test_split_k_decode_llama70b(li):
     ref, absref = oracle.linear_entries(oracle.FWD, rqx, fx, rbx, rqw, fw, rbw, T,
                                         lin.in_features, lin.out_features, rows, cols)
     assert_gemm_close(to_f64(y)[rows, cols], ref, absref, "decode %s" % lin.name)
+
+
+def test_plan_query_errors():
+    with pytest.raises(fp8.Fp8Error) as e:
+        fp8.fp8_linear_plan(7, 16, 16, 16)
+    assert e.value.status == 1
+    with pytest.raises(fp8.Fp8Error):
+        fp8.fp8_linear_plan(fp8.FWD, -1, 16, 16)
+    # decode-sized forward without a workspace: narrow 128 x 64 tiles
+    assert fp8.fp8_linear_plan(fp8.FWD, 16, 8192, 8192)["tile_n"] == 64
 
 
 def test_split_k_workspace_errors():
@@ -377,3 +389,67 @@ def test_step_graph_replay_matches_eager():
             [(inputs[0][0][:16, :16].contiguous(), inputs[0][1][:16, :16].contiguous(),
               inputs[0][2][:16, :16].contiguous())])
 
+
+@pytest.mark.parametrize("T,In,Out", [(8192, 768, 768), (4096, 512, 256), (3000, 256, 640)])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_split_k_small_weight_gradient(T, In, Out, out_dtype):
+    """Small dW over many tokens: CTA-pair tiles split along K (T) through the
+    workspace entry point, full oracle comparison, deterministic."""
+    assert fp8.fp8_linear_bwd_wgrad_workspace_size(T, In, Out) > 0
+    plan = fp8.fp8_linear_plan(fp8.WGRAD, T, In, Out, with_workspace=True)
+    assert plan["ctas_per_tile"] == 2 and plan["k_splits"] > 1, plan
+    assert fp8.fp8_linear_plan(fp8.WGRAD, T, In, Out)["k_splits"] == 1
+    x, w, dy = _inputs(T, In, Out, seed=T + In + Out)
+    Q = _passes(x, w, dy)
+    qx, bx, rqx, rbx, fx = Q["x"]
+    qdy, bdy, rqdy, rbdy, fdy = Q["dy"]
+    a = fp8.fp8_linear_bwd_wgrad_ws(qdy, fdy, bdy, qx, fx, bx, out_dtype=out_dtype)
+    b = fp8.fp8_linear_bwd_wgrad_ws(qdy, fdy, bdy, qx, fx, bx, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    ref, absref = oracle.linear(oracle.WGRAD, rqdy, fdy, rbdy, rqx, fx, rbx, T, In, Out)
+    assert_gemm_close(to_f64(a), ref, absref, "split-K wgrad %s" % ((T, In, Out),))
+
+
+# Problems of many tiles run on 256 x 512 CTA-pair tiles (two M=256, N=256
+# MMAs per K step sharing the A stage, one 512-column accumulator drained in
+# two halves).  The shapes below are in that regime and ragged in every
+# dimension: 9 row blocks (the last one partly filled); N = 8000 leaves 320
+# columns in the last 512-column block (64 in its second half), N = 7696
+# leaves 16 (its second half empty: neither loaded nor multiplied); K ragged
+# against the 128-wide k-blocks.  Every element of rows and columns at the
+# tile and half-tile edges is checked, plus random samples.
+@pytest.mark.parametrize("N", [8000, 7696])
+@pytest.mark.parametrize("pass_", [oracle.FWD, oracle.DGRAD, oracle.WGRAD])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_double_width_tiles(N, pass_, out_dtype):
+    if pass_ == oracle.FWD:
+        T, In, Out = 2148, 400, N
+    elif pass_ == oracle.DGRAD:
+        T, In, Out = 2148, N, 400
+    else:
+        T, In, Out = 300, N, 2160
+    plan = fp8.fp8_linear_plan(pass_, T, In, Out)
+    assert (plan["tile_m"], plan["tile_n"], plan["ctas_per_tile"], plan["k_splits"]) == \
+        (256, 512, 2, 1), plan
+    x, w, dy = _inputs(T, In, Out, seed=N + 10 * pass_)
+    Q = _passes(x, w, None if pass_ == oracle.FWD else dy)
+    y = _run(pass_, Q, out_dtype)
+    torch.cuda.synchronize()
+    R, C = y.shape
+    edge_rows = sorted({0, 1, 127, 128, 255, 256, R - 101, R - 100, R - 1})
+    last = (C - 1) // 512 * 512
+    edge_cols = sorted({0, 31, 32, 255, 256, 511, 512, last - 1, last, last + 255, last + 256,
+                        C - 1} & set(range(C)))
+    rng = np.random.default_rng(N + pass_)
+    parts_r = [rng.integers(0, R, 1 << 14)]
+    parts_c = [rng.integers(0, C, 1 << 14)]
+    for r in edge_rows:
+        parts_r.append(np.full(C, r))
+        parts_c.append(np.arange(C))
+    for c in edge_cols:
+        parts_r.append(np.arange(R))
+        parts_c.append(np.full(R, c))
+    rows, cols = np.concatenate(parts_r), np.concatenate(parts_c)
+    ref, absref = oracle.linear_entries(pass_, *_oracle_args(pass_, Q), T, In, Out, rows, cols)
+    assert_gemm_close(to_f64(y)[rows, cols], ref, absref, "double tile pass %d %s" % (pass_, (T, In, Out)))

@@ -49,7 +49,11 @@ def _call_noalloc(qx, bx, qw, bw, y):
              y.data_ptr(), fp8.BF16 if y.dtype == torch.bfloat16 else fp8.FP32, c.c_void_p(stream))
 
 
-@pytest.mark.parametrize("T,In,Out,splits", [(16, 12288, 512, True), (200, 512, 384, False)])
+# (16, 12288, 512): 128-row tiles split K; (1024, 8192, 256): CTA-pair tiles
+# split K within the scratch; (2048, 2048, 1024): a pair split would need more
+# than the scratch holds, so the forward runs unsplit; (200, 512, 384): no split
+@pytest.mark.parametrize("T,In,Out,splits", [(16, 12288, 512, True), (1024, 8192, 256, True),
+                                             (2048, 2048, 1024, True), (200, 512, 384, False)])
 @pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
 def test_noalloc_matches_workspace_entry_point(T, In, Out, splits, out_dtype):
     assert (fp8.fp8_linear_fwd_workspace_size(T, In, Out) > 0) == splits
