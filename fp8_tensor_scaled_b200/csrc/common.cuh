@@ -74,6 +74,32 @@ __device__ __forceinline__ void tma_load_2d(uint32_t smem_dst, const void* desc,
       : "memory");
 }
 
+// TMA store of a 2-D box from this CTA's shared memory (bulk-group
+// completion).  Coordinates are non-negative; the box is clipped at the
+// tensor's bounds.
+__device__ __forceinline__ void tma_store_2d(const void* desc, uint32_t smem_src, int32_t x,
+                                             int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];"
+      ::"l"(reinterpret_cast<uint64_t>(desc)), "r"(smem_src), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the shared memory of every committed bulk store may be overwritten
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// every committed bulk store has completed
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// generic-proxy writes to shared memory become visible to the async proxy (TMA)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory, MMA, commit, loads, fences
 // ---------------------------------------------------------------------------

@@ -139,9 +139,17 @@ template <int kTile> constexpr uint32_t tmem_cols() {
   return kTile == kTileDouble ? 512u : 2u * Cfg<kTile>::BN;
 }
 template <int kTile> constexpr int num_bars() { return 2 * Cfg<kTile>::STAGES + 2 + 2 + 1; }
+// Epilogue staging for the TMA store of D: per epilogue warp, 32 rows x 128
+// bytes, twice (two 32-column fp32 boxes or one 64-column BF16 box).
+constexpr uint32_t kStageOutBytesPerWarp = 2 * 32 * 128;
+constexpr uint32_t kStageOutBytes = 4 * kStageOutBytesPerWarp;   // 32 KB
 template <int kTile> constexpr size_t smem_bytes() {
-  return 1024 + Cfg<kTile>::STAGES * stage_bytes<kTile>() + num_bars<kTile>() * 8 + 16;
+  return 1024 + Cfg<kTile>::STAGES * stage_bytes<kTile>() + kStageOutBytes +
+         num_bars<kTile>() * 8 + 16;
 }
+static_assert(smem_bytes<kTileSingle>() <= 232448 && smem_bytes<kTilePair>() <= 232448 &&
+                  smem_bytes<kTileNarrow>() <= 232448 && smem_bytes<kTileDouble>() <= 232448,
+              "227 KB of shared memory per block");
 
 struct Params {
   int M, N, K;
@@ -221,53 +229,51 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
-// Scale, round and store one row's 32 consecutive accumulator columns
-// (fp32 bits in r) at D[row, col0 ..]; with kAmax also fold max |stored| into
-// dmax (fp32 bits, or two packed bf16 maxima).
+// Scale and round one row's 64 accumulator columns (fp32 bits: r0 = columns
+// 0..31, r1 = 32..63) and write them to the warp's staging buffer at `stage`
+// (row `lane`, 128-byte rows, 128-byte swizzle: 16-byte piece j of a row
+// goes to piece j ^ (lane % 8)).  BF16: one 64-column box of 128-byte rows.
+// FP32: two 32-column boxes, the second 4 KB after the first.  With kAmax
+// also fold max |stored| into dmax.
 template <bool kOutF32, bool kAmax>
-__device__ __forceinline__ void store_row_chunk(const Params& p, int64_t row, int col0,
-                                                const uint32_t (&r)[32], const Pow2Scale& sc,
-                                                uint32_t& dmax) {
+__device__ __forceinline__ void stage_out_chunks(uint32_t stage, int lane, const uint32_t (&r0)[32],
+                                                 const uint32_t (&r1)[32], const Pow2Scale& sc,
+                                                 uint32_t& dmax) {
+  const uint32_t row_base = stage + static_cast<uint32_t>(lane) * 128u;
+  const uint32_t sw = static_cast<uint32_t>(lane & 7);
   if (kOutF32) {
-    float* dst = static_cast<float*>(p.d) + row * p.N + col0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (col0 + 4 * j < p.N) {
-        float4 v;
-        v.x = apply_pow2(__uint_as_float(r[4 * j + 0]), sc);
-        v.y = apply_pow2(__uint_as_float(r[4 * j + 1]), sc);
-        v.z = apply_pow2(__uint_as_float(r[4 * j + 2]), sc);
-        v.w = apply_pow2(__uint_as_float(r[4 * j + 3]), sc);
-        *reinterpret_cast<float4*>(dst + 4 * j) = v;
-        if (kAmax)
-          dmax = max(dmax, max(max(__float_as_uint(v.x) & 0x7FFFFFFFu,
-                                   __float_as_uint(v.y) & 0x7FFFFFFFu),
-                               max(__float_as_uint(v.z) & 0x7FFFFFFFu,
-                                   __float_as_uint(v.w) & 0x7FFFFFFFu)));
+    for (int b = 0; b < 2; ++b) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t bits = b == 0 ? r0[4 * j + e] : r1[4 * j + e];
+          w[e] = __float_as_uint(apply_pow2(__uint_as_float(bits), sc));
+          if (kAmax) dmax = max(dmax, w[e] & 0x7FFFFFFFu);
+        }
+        const uint32_t addr = row_base + static_cast<uint32_t>(b) * 4096u +
+                              ((static_cast<uint32_t>(j) ^ sw) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                     ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
       }
     }
   } else {
-    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.d) + row * p.N + col0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (col0 + 8 * j < p.N) {
-        uint4 v;
-        v.x = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 0]), sc),
-                          apply_pow2(__uint_as_float(r[8 * j + 1]), sc));
-        v.y = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 2]), sc),
-                          apply_pow2(__uint_as_float(r[8 * j + 3]), sc));
-        v.z = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 4]), sc),
-                          apply_pow2(__uint_as_float(r[8 * j + 5]), sc));
-        v.w = pack_bf16x2(apply_pow2(__uint_as_float(r[8 * j + 6]), sc),
-                          apply_pow2(__uint_as_float(r[8 * j + 7]), sc));
-        *reinterpret_cast<uint4*>(dst + 8 * j) = v;
-        if (kAmax) {
-          dmax = __vmaxu2(dmax, v.x & 0x7FFF7FFFu);
-          dmax = __vmaxu2(dmax, v.y & 0x7FFF7FFFu);
-          dmax = __vmaxu2(dmax, v.z & 0x7FFF7FFFu);
-          dmax = __vmaxu2(dmax, v.w & 0x7FFF7FFFu);
-        }
+    for (int j = 0; j < 8; ++j) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int col = 8 * j + 2 * e;          // 0..63
+        const uint32_t lo = col < 32 ? r0[col] : r1[col - 32];
+        const uint32_t hi = col < 32 ? r0[col + 1] : r1[col - 31];
+        w[e] = pack_bf16x2(apply_pow2(__uint_as_float(lo), sc), apply_pow2(__uint_as_float(hi), sc));
+        if (kAmax) dmax = __vmaxu2(dmax, w[e] & 0x7FFF7FFFu);
       }
+      const uint32_t addr = row_base + ((static_cast<uint32_t>(j) ^ sw) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                   ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
     }
   }
 }
@@ -279,7 +285,8 @@ __device__ __forceinline__ void store_row_chunk(const Params& p, int64_t row, in
 template <int kTile, bool kAMN, bool kBMN, bool kOutF32, bool kAmax>
 __global__ void __launch_bounds__(kThreads, 1)
 fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                const __grid_constant__ CUtensorMap tmap_b, const Params p) {
+                const __grid_constant__ CUtensorMap tmap_b,
+                const __grid_constant__ CUtensorMap tmap_d, const Params p) {
   using C = Cfg<kTile>;
   constexpr int kCta = C::CTAS;
   constexpr int BN = C::BN;
@@ -299,7 +306,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sOut = smem + STAGES * STAGE_BYTES;                 // 1024-byte aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + kStageOutBytes);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -331,6 +339,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     fence_mbarrier_init();
     tma_prefetch_desc(&tmap_a);
     tma_prefetch_desc(&tmap_b);
+    tma_prefetch_desc(&tmap_d);
   }
   if (warp == 1) {
     if (kCta == 2) {
@@ -519,6 +528,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     // ------------------------------- epilogue -------------------------------
     const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
     const int row_in_tile = static_cast<int>(rank) * 128 + quarter * 32 + lane;
+    const uint32_t out_stage = smem_u32(sOut) + static_cast<uint32_t>(warp - 2) * kStageOutBytesPerWarp;
     const Pow2Scale sc = make_pow2_scale(-(*p.bias_a + *p.bias_b));
     uint32_t dmax = 0;   // kAmax: this thread's max |D| bits (packed bf16 pair or fp32)
     int local = 0;
@@ -538,6 +548,8 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       tile_coords(t, p, mb, nb);
       const int64_t row = static_cast<int64_t>(mb) * C::BM + row_in_tile;
       const bool row_ok = row < p.M;
+      // first row of this warp's 32-row box of D
+      const int row_box = mb * C::BM + static_cast<int>(rank) * 128 + quarter * 32;
       if (!kDbl && p.splits > 1) {
         // ---- split K: store this range's raw fp32 partial and free the
         // accumulator; splitk_reduce_kernel sums the ranges afterwards
@@ -572,7 +584,13 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       static_assert(kChunks % 2 == 0, "chunks are drained in pairs");
 #pragma unroll 1
       for (int h = 0; h < kHalves; ++h) {
-        // two 32-column loads in flight per wait (kChunks is even)
+        // Two 32-column TMEM loads in flight per wait (kChunks is even).
+        // The 64 columns are scaled, rounded and written to this warp's
+        // staging buffer in the 128-byte-swizzled layout of the D tensor
+        // map's box (row = lane; 16-byte piece j of a 128-byte row at
+        // j ^ (row % 8)), then stored by one TMA store (BF16: one 64-column
+        // box; FP32: two 32-column boxes).  Rows and columns outside D are
+        // clipped by the TMA unit.
 #pragma unroll 1
         for (int c = h * kChunks; c < (h + 1) * kChunks; c += 2) {
           const int col0 = nb * BN + c * 32;
@@ -583,10 +601,21 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
           uint32_t r0[32], r1[32];
           tmem_ld_32x32b_x32(taddr, r0);
           if (two) tmem_ld_32x32b_x32(taddr + 32u, r1);
+          else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r1[j] = 0u;
+          }
+          // the staging buffer is free once the previous stores have read it
+          if (lane == 0) bulk_wait_group_read0();
+          __syncwarp();
           tmem_ld_wait();
-          if (row_ok) {
-            store_row_chunk<kOutF32, kAmax>(p, row, col0, r0, sc, dmax);
-            if (two) store_row_chunk<kOutF32, kAmax>(p, row, col0 + 32, r1, sc, dmax);
+          stage_out_chunks<kOutF32, kAmax>(out_stage, lane, r0, r1, sc, dmax);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row_box < p.M) {
+            tma_store_2d(&tmap_d, out_stage, col0, row_box);
+            if (kOutF32 && two) tma_store_2d(&tmap_d, out_stage + 4096u, col0 + 32, row_box);
+            bulk_commit_group();
           }
         }
         // these columns are free for the next tile's MMAs
@@ -599,6 +628,9 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
       }
     }
+    // every TMA store of this warp has completed before the block can exit
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
     if (kAmax) {
       // a bf16 is the top half of an fp32: widen the packed pair's max
       uint32_t bits = kOutF32 ? dmax : (max(dmax & 0xFFFFu, dmax >> 16) << 16);
@@ -726,6 +758,22 @@ bool encode_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D row-major D [rows, cols] (BF16 or FP32) for the epilogue's TMA stores:
+// box of 128 bytes (64 BF16 / 32 FP32 columns) x 32 rows, 128-byte swizzle.
+bool encode_out_2d(CUtensorMap* m, const void* ptr, bool fp32, uint64_t cols, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t esz = fp32 ? 4 : 2;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * esz};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int g_sm_count[64];
 
 int sm_count() {
@@ -823,7 +871,9 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
   const bool ok_a = kAMN ? encode_2d(&ta, g.a, M, K, 128, BK) : encode_2d(&ta, g.a, K, M, BK, 128);
   const bool ok_b = kBMN ? encode_2d(&tb, g.b, N, K, 128, BK)
                          : encode_2d(&tb, g.b, K, N, BK, b_box_rows);
-  if (!ok_a || !ok_b) return FP8_ERR_CUDA;
+  CUtensorMap td;
+  const bool ok_d = encode_out_2d(&td, g.d, g.d_fp32, N, M);
+  if (!ok_a || !ok_b || !ok_d) return FP8_ERR_CUDA;
 
   Params p;
   p.M = static_cast<int>(g.M);
@@ -902,7 +952,7 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
   }
   const int units = p.num_work < max_units[dev] ? p.num_work : max_units[dev];
   cfg.gridDim = dim3(static_cast<unsigned>(units * kCta), 1, 1);
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, p) != cudaSuccess) return FP8_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, td, p) != cudaSuccess) return FP8_ERR_CUDA;
   if (p.splits > 1) {
     const int64_t n4 = static_cast<int64_t>(g.M) * g.N / 4;
     int64_t blocks = (n4 + kReduceThreads - 1) / kReduceThreads;
