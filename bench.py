@@ -210,7 +210,16 @@ class Workload:
         self.cast_only_bytes = sum((t.element_size() + 1) * t.numel()
                                    for inp in self.inputs for t in inp)
         self.bias_every = bias_every
-        self.kernels_per_step = len(self.layers) * (3 * 2 + 3)   # 3 x (amax + cast) + 3 GEMMs
+        # kernels of one step: per linear 3 casts, 3 amax passes on bias-refresh
+        # steps, 3 GEMMs, and the split-K reduction of a wgrad that splits
+        self.gemm_kernels_per_step = sum(
+            3 + (1 if l.wgrad_ws is not None and fp8.fp8_linear_plan(
+                fp8.WGRAD, l.T, l.inf, l.outf, with_workspace=True)["k_splits"] > 1 else 0)
+            for l in self.layers)
+
+    def launches(self, refresh_steps, steps):
+        n = len(self.layers)
+        return steps * (self.gemm_kernels_per_step + 3 * n) + refresh_steps * 3 * n
 
     def new_timing(self):
         n = len(self.layers)
@@ -256,7 +265,7 @@ def run_fp8(args, world, rank, local):
                    + (args.steps - refresh_steps) * wl.cast_only_bytes)
     res = dict(ms=ms, ms_local=ms_local, quant_ms=quant_ms, gemm_ms=gemm_ms,
                per_linear_gemm_ms=per_linear_gemm_ms, clocks=clocks, wl=wl,
-               quant_bytes=quant_bytes)
+               quant_bytes=quant_bytes, launches=wl.launches(refresh_steps, args.steps))
     if args.graph:
         wl.stepper.capture(wl.inputs)
         for _ in range(max(3, args.warmup)):
@@ -274,6 +283,7 @@ def run_fp8(args, world, rank, local):
         barrier(world)
         res["ms_eager"] = ms
         res["ms"] = max_over_ranks(world, start.elapsed_time(end), device)
+        res["launches"] = wl.launches(args.steps, args.steps)   # captured with refresh
 
     if not args.no_e2e:
         res["e2e"] = run_e2e(args, wl, device, world)
@@ -566,7 +576,7 @@ def main():
                            "kernel": "amax_kernel + cast_kernel",
                            "bytes_per_element": "2*s_in + 1", "peak_source": peak_src},
         "clocks": r["clocks"],
-        "gpu_launches": wl.kernels_per_step * steps,
+        "gpu_launches": r["launches"],
     }
     if "ms_eager" in r:
         line["ms_per_step_eager"] = round(r["ms_eager"] / steps, 4)

@@ -132,6 +132,10 @@ template <> struct Cfg<kTileDouble> {
   static constexpr int CTAS = 2, BM = 256, BN = 512, MMA_N = 256, B_ROWS = 256, STAGES = 4;
 };
 constexpr uint32_t B_HALF_BYTES = 128 * BK;   // 16 KB: one 128-row B box
+// Double-width tile: stages of a new tile multiplied into the first half of
+// the accumulator only, while the epilogue still drains the second half
+// (1 <= kDeferStages <= the ring depth).
+constexpr int kDeferStages = 4;
 template <int kTile> constexpr uint32_t b_bytes() { return Cfg<kTile>::B_ROWS * BK; }
 template <int kTile> constexpr uint32_t stage_bytes() { return A_BYTES + b_bytes<kTile>(); }
 // two fp32 accumulators of BN columns each; the wide tile has one of 512
@@ -452,7 +456,7 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
       // producer can fill).  The rest run both halves stage by stage.
       int defer = 0;
       if (kDbl) {
-        defer = min(STAGES, kb1 - kb0);
+        defer = min(kDeferStages, kb1 - kb0);
         int st = stage;
         uint32_t ph = phase;
         for (int i = 0; i < defer; ++i) {

@@ -63,45 +63,68 @@ class Fp8AmaxLinear:
             if ws > 0:
                 self.wgrad_ws = torch.empty(ws, **u8)
 
-    def quantize(self, x, w, dy=None):
-        """Cast X, W (E4M3) and dY (E5M2).  On refresh steps amax -> bias ->
-        cast (fp8_quantize); otherwise cast with the stored bias."""
+    # tensor indices (amax / bias slots) and pass indices
+    X, W, DY = 0, 1, 2
+    FWD, DGRAD, WGRAD = 0, 1, 2
+    # the quantized tensors each pass reads
+    PASS_INPUTS = {FWD: (X, W), DGRAD: (DY, W), WGRAD: (DY, X)}
+
+    def begin_step(self):
+        """Start a step: returns whether it recomputes amax and bias (refresh)
+        or casts with the stored biases."""
         refresh = self.fixed is None and self.calls % self.every == 0
         self.calls += 1
-        work = [(x, E4M3, 0, self.x8), (w, E4M3, 1, self.w8)]
+        return refresh
+
+    def quantize_one(self, i, t, refresh):
+        """Cast tensor i (X or W to E4M3, dY to E5M2) on the current stream.
+        On refresh steps amax -> bias -> cast (fp8_quantize); otherwise cast
+        with the stored bias."""
+        fmt = E5M2 if i == self.DY else E4M3
+        out = (self.x8, self.w8, self.dy8)[i]
+        if refresh:
+            fp8_quantize(t, fmt, self.margins[i], self.amax[i:i + 1], self.bias[i:i + 1], out)
+        else:
+            fp8_cast_scaled(t, self.bias[i:i + 1], fmt, out=out)
+
+    def quantize(self, x, w, dy=None):
+        """Cast X, W (E4M3) and dY (E5M2)."""
+        refresh = self.begin_step()
+        self.quantize_one(self.X, x, refresh)
+        self.quantize_one(self.W, w, refresh)
         if self.backward:
-            work.append((dy, E5M2, 2, self.dy8))
-        for t, fmt, i, out in work:
-            if refresh:
-                fp8_quantize(t, fmt, self.margins[i], self.amax[i:i + 1], self.bias[i:i + 1], out)
-            else:
-                fp8_cast_scaled(t, self.bias[i:i + 1], fmt, out=out)
+            self.quantize_one(self.DY, dy, refresh)
+
+    def gemm(self, k):
+        """One pass on the current stream: FWD (Y), DGRAD (dX) or WGRAD (dW)."""
+        bx, bw, bdy = self.bias[0:1], self.bias[1:2], self.bias[2:3]
+        if k == self.FWD:
+            fp8_linear_fwd(self.x8, E4M3, bx, self.w8, E4M3, bw, out=self.y)
+        elif k == self.DGRAD:
+            fp8_linear_bwd_dgrad(self.dy8, E5M2, bdy, self.w8, E4M3, bw, out=self.dx)
+        elif self.wgrad_ws is not None:
+            fp8_linear_bwd_wgrad_ws(self.dy8, E5M2, bdy, self.x8, E4M3, bx, out=self.dw,
+                                    workspace=self.wgrad_ws)
+        else:
+            fp8_linear_bwd_wgrad(self.dy8, E5M2, bdy, self.x8, E4M3, bx, out=self.dw)
+
+    def outputs(self):
+        return (self.y, self.dx, self.dw) if self.backward else (self.y,)
 
     def gemms(self, pass_done=None):
-        """The three GEMMs on the current stream.  `pass_done` (optional): one
+        """The passes on the current stream.  `pass_done` (optional): one
         CUDA event per pass (fwd, dgrad, wgrad), each recorded as soon as that
         pass's output is complete, so a consumer can take Y before dX and dW
         are done."""
-        bx, bw, bdy = self.bias[0:1], self.bias[1:2], self.bias[2:3]
-        fp8_linear_fwd(self.x8, E4M3, bx, self.w8, E4M3, bw, out=self.y)
-        if pass_done is not None:
-            pass_done[0].record()
-        if self.backward:
-            fp8_linear_bwd_dgrad(self.dy8, E5M2, bdy, self.w8, E4M3, bw, out=self.dx)
+        for k in ((self.FWD, self.DGRAD, self.WGRAD) if self.backward else (self.FWD,)):
+            self.gemm(k)
             if pass_done is not None:
-                pass_done[1].record()
-            if self.wgrad_ws is not None:
-                fp8_linear_bwd_wgrad_ws(self.dy8, E5M2, bdy, self.x8, E4M3, bx, out=self.dw,
-                                        workspace=self.wgrad_ws)
-            else:
-                fp8_linear_bwd_wgrad(self.dy8, E5M2, bdy, self.x8, E4M3, bx, out=self.dw)
-            if pass_done is not None:
-                pass_done[2].record()
+                pass_done[k].record()
 
     def step(self, x, w, dy=None):
         self.quantize(x, w, dy)
         self.gemms()
-        return (self.y, self.dx, self.dw) if self.backward else (self.y,)
+        return self.outputs()
 
     def flops(self):
         return 2 * self.T * self.inf * self.outf * (3 if self.backward else 1)
@@ -125,10 +148,10 @@ class Fp8AmaxStep:
         graph (on these input and output buffers) and replayed with a single
         host call: no per-kernel launch cost, which matters for small layers.
     ``step_from_host(h_in, d_in, h_out)``  the same step from pinned host tensors:
-        copies in on one copy stream, copies of each linear's Y, dX, dW out on
-        another as soon as the pass that writes it finishes, so transfers in both directions
-        overlap each other and the compute.  Returns when the caller's stream
-        has been ordered after the last copy out.
+        copies in on one copy stream and out on another, scheduled per tensor
+        and per pass so that transfers in both directions overlap each other
+        and the compute.  Returns when the caller's stream has been ordered
+        after the last copy out.
     """
 
     def __init__(self, linears, overlap=True):
@@ -141,9 +164,10 @@ class Fp8AmaxStep:
         self.d2h = torch.cuda.Stream(dev)
         n = len(self.linears)
         self.q_done = [torch.cuda.Event() for _ in range(n)]
-        self.in_done = [torch.cuda.Event() for _ in range(n)]
         self.g_done = [torch.cuda.Event() for _ in range(n)]
         self.p_done = [[torch.cuda.Event() for _ in range(3)] for _ in range(n)]
+        self.t_in = [[torch.cuda.Event() for _ in range(3)] for _ in range(n)]
+        self.t_q = [[torch.cuda.Event() for _ in range(3)] for _ in range(n)]
         self.out_done = torch.cuda.Event()
 
     def flops(self):
@@ -204,23 +228,76 @@ class Fp8AmaxStep:
     def replay(self):
         self.graph.replay()
 
+    def host_plan(self):
+        """Schedule of the host-buffer step: [(linear, input arrival order,
+        pass order), ...].
+
+        The copy out of a pass's output can start only once both of its inputs
+        are in, so the copies out trail the copies in at the start of the step
+        (the head) and outlast them at the end (the tail: the outputs that
+        depend on the last input to arrive).  Per linear the input whose
+        dependent outputs are the fewest bytes arrives last, and the pass that
+        does not need it runs first; the linear whose first pass needs the
+        fewest input bytes goes first, the one with the smallest tail last."""
+        L = Fp8AmaxLinear
+        plans = []
+        for i, l in enumerate(self.linears):
+            if not l.backward:
+                plans.append((i, (L.W, L.X), (L.FWD,), l.T * l.inf + l.outf * l.inf, 0))
+                continue
+            ins = {L.X: l.T * l.inf, L.W: l.outf * l.inf, L.DY: l.T * l.outf}
+            outs = {L.FWD: l.T * l.outf, L.DGRAD: l.T * l.inf, L.WGRAD: l.outf * l.inf}
+            deps = {t: [k for k in outs if t in L.PASS_INPUTS[k]] for t in ins}
+            last = min(ins, key=lambda t: (sum(outs[k] for k in deps[t]), t))
+            first_pass = next(k for k in outs if last not in L.PASS_INPUTS[k])
+            arrival = tuple(t for t in L.PASS_INPUTS[first_pass]) + (last,)
+            passes = (first_pass,) + tuple(k for k in (L.FWD, L.DGRAD, L.WGRAD) if k != first_pass)
+            head = sum(ins[t] for t in L.PASS_INPUTS[first_pass])
+            tail = sum(outs[k] for k in deps[last])
+            plans.append((i, arrival, passes, head, tail))
+        first = min(plans, key=lambda q: (q[3], q[0]))
+        rest = [q for q in plans if q is not first]
+        if rest:
+            last = min(rest, key=lambda q: (q[4], -q[0]))
+            rest = [q for q in rest if q is not last] + [last]
+        return [(q[0], q[1], q[2]) for q in [first] + rest]
+
     def step_from_host(self, host_inputs, device_inputs, host_outputs):
+        """One step from pinned host tensors host_inputs[i] = (x, w, dy) into
+        the device buffers device_inputs[i], results copied to host_outputs[i]
+        = (y, dx, dw).  The copies in run on one stream in the order of
+        host_plan(); each tensor is quantized as soon as it has arrived; each
+        pass runs as soon as its two operands are quantized; each output
+        leaves on a second copy stream as soon as its pass is done."""
         main = torch.cuda.current_stream(self.device)
+        qs = self.side if self.overlap else main
         start = torch.cuda.Event()
         start.record(main)
+        self.h2d.wait_event(start)          # device inputs free: the previous step is done
+        plans = [(i, self.linears[i], arrival, passes) for i, arrival, passes in self.host_plan()]
+        L = Fp8AmaxLinear
         with torch.cuda.stream(self.h2d):
-            self.h2d.wait_event(start)       # device inputs free: the previous step is done
-            for i, (hs, ds) in enumerate(zip(host_inputs, device_inputs)):
-                for h, d in zip(hs, ds):
-                    d.copy_(h, non_blocking=True)
-                self.in_done[i].record(self.h2d)
-        self.step(device_inputs, in_events=self.in_done)
+            for i, lin, tensors, _ in plans:
+                for t in tensors:
+                    device_inputs[i][t].copy_(host_inputs[i][t], non_blocking=True)
+                    self.t_in[i][t].record(self.h2d)
+        for i, lin, tensors, passes in plans:
+            refresh = lin.begin_step()
+            with torch.cuda.stream(qs):
+                for t in tensors:
+                    qs.wait_event(self.t_in[i][t])
+                    lin.quantize_one(t, device_inputs[i][t], refresh)
+                    self.t_q[i][t].record(qs)
+            for k in passes:
+                for t in L.PASS_INPUTS[k]:
+                    main.wait_event(self.t_q[i][t])
+                lin.gemm(k)
+                self.p_done[i][k].record(main)
         with torch.cuda.stream(self.d2h):
-            # each output leaves as soon as its own pass is done: the copy of
-            # Y overlaps dgrad and wgrad, so the last copy out starts earlier
-            for i, (lin, hs) in enumerate(zip(self.linears, host_outputs)):
-                for k, (h, d) in enumerate(zip(hs, (lin.y, lin.dx, lin.dw))):
+            for i, lin, _, passes in plans:
+                outs = lin.outputs()
+                for k in passes:
                     self.d2h.wait_event(self.p_done[i][k])
-                    h.copy_(d, non_blocking=True)
+                    host_outputs[i][k].copy_(outs[k], non_blocking=True)
             self.out_done.record(self.d2h)
         main.wait_event(self.out_done)

@@ -340,6 +340,34 @@ def test_split_k_decode_llama70b(li):
     assert_gemm_close(to_f64(y)[rows, cols], ref, absref, "decode %s" % lin.name)
 
 
+def test_step_from_host_matches_device_step():
+    """The host-buffer step (copies in and out scheduled per tensor and per
+    pass, linears reordered) gives the device-resident step's results bit for
+    bit, and the biases of every linear."""
+    from fp8_tensor_scaled_b200.layer import Fp8AmaxStep
+    shapes = [(256, 384, 512), (256, 128, 256), (256, 512, 384)]
+    dev_l, host_l, inputs = [], [], []
+    for i, (T, In, Out) in enumerate(shapes):
+        x, w, dy = _inputs(T, In, Out, seed=70 + i)
+        inputs.append((x, w, dy))
+        dev_l.append(fp8.Fp8AmaxLinear(T, In, Out, DEV))
+        host_l.append(fp8.Fp8AmaxLinear(T, In, Out, DEV))
+    d_in = [tuple(t.to(DEV) for t in inp) for inp in inputs]
+    scratch = [tuple(torch.empty_like(t) for t in inp) for inp in d_in]
+    h_in = [tuple(t.pin_memory() for t in inp) for inp in inputs]
+    h_out = [tuple(torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in l.outputs())
+             for l in host_l]
+    a, b = Fp8AmaxStep(dev_l), Fp8AmaxStep(host_l)
+    for _ in range(2):
+        a.step(d_in)
+        b.step_from_host(h_in, scratch, h_out)
+    torch.cuda.synchronize()
+    for la, lb, ho in zip(dev_l, host_l, h_out):
+        assert torch.equal(la.bias, lb.bias)
+        for o, h in zip(la.outputs(), ho):
+            assert torch.equal(o.cpu(), h)
+
+
 def test_plan_query_errors():
     with pytest.raises(fp8.Fp8Error) as e:
         fp8.fp8_linear_plan(7, 16, 16, 16)
