@@ -2,7 +2,7 @@
 """Benchmark of the FP8-AMAX linear layer on B200: one JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fp8amax|reference]
-                    [--workload c3|c2|c1] [--no-e2e] [--no-cpu-baseline]
+                    [--workload c3|c2|c1|c4|decode] [--graph] [--no-e2e] [--no-cpu-baseline]
 
 A step is one pass of the whole hot path over the Llama-2-70B-shaped workload
 (d 8192, ffn 28672, GQA QKV 8192->10240, 8192 tokens): for each of the four
@@ -17,6 +17,11 @@ pinned HOST buffers: each step copies X, W, dY in and Y, dX, dW back.  The
 `roofline` object is the dominant kernel (the FP8 GEMM) against the dense FP8
 tensor-core peak; `roofline_quant` the amax+cast kernels against HBM.
 `cpu_baseline` is the CPU oracle timed on a bounded sample of the same step.
+
+Other workloads (each its own JSON line): c1 / c2 the GPT-111M and
+Llama-2-7B layer shapes; c4 the amax + bias + cast of one tensor
+(`--sweep-log2n`, `--sweep-dtype`); decode the Llama-2-70B projections'
+forward for `--decode-tokens` tokens with the weights cast once.
 
 With N > 1 (torchrun, one process per GPU) every rank runs its own replica of
 the step (the layer does not shard across GPUs here): weak scaling, `value` =
@@ -50,9 +55,12 @@ def parse():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="fp8amax", choices=["fp8amax", "reference"])
-    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4"],
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "decode"],
                     help="c3: the Llama-2-70B projections (default); c1/c2: smaller layer "
-                         "shapes; c4: the amax+bias+cast sweep alone on one tensor")
+                         "shapes; c4: the amax+bias+cast sweep alone on one tensor; decode: "
+                         "the forward of the Llama-2-70B projections for few tokens, weights "
+                         "cast once (inference)")
+    ap.add_argument("--decode-tokens", type=int, default=16, help="decode: tokens per forward")
     ap.add_argument("--sweep-log2n", type=int, default=28, help="c4: log2 of the element count")
     ap.add_argument("--sweep-dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -332,6 +340,80 @@ def run_sweep(args, world, rank, local):
     return 0
 
 
+def run_decode(args, world, rank, local):
+    """Inference forward of the Llama-2-70B projections for a few tokens: the
+    weights are cast to E4M3 once (outside the timed region, as a deployed
+    model holds them), each step quantizes X (amax + bias + cast) and runs
+    Y = X8 . W8^T for every projection through fp8_linear_fwd_ws (split K
+    with a workspace).  Bound by HBM: the step streams every weight once.
+    L2 is flushed before each step; the flush is outside the timed region."""
+    import fp8_tensor_scaled_b200 as fp8
+    device = torch.device("cuda", local)
+    cfg = workloads.C3
+    T = args.decode_tokens
+    layers = []
+    for li, lin in enumerate(cfg.linears):
+        x, w, _ = workloads.linear_inputs(3, li, device=device)
+        _, bw, w8 = fp8.fp8_quantize(w, fp8.E4M3, 0)
+        del w
+        x = x[:T].contiguous()
+        need = fp8.fp8_linear_fwd_workspace_size(T, lin.in_features, lin.out_features)
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+        y = torch.empty((T, lin.out_features), dtype=torch.bfloat16, device=device)
+        amax = torch.empty(1, dtype=torch.float32, device=device)
+        bx = torch.empty(1, dtype=torch.int32, device=device)
+        x8 = torch.empty((T, lin.in_features), dtype=torch.uint8, device=device)
+        layers.append((lin, x, x8, amax, bx, w8, bw, y, ws, need))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)     # 2 x L2
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for lin, x, x8, amax, bx, w8, bw, y, ws, need in layers:
+            fp8.fp8_quantize(x, fp8.E4M3, 0, amax, bx, x8)
+            fp8.fp8_linear_fwd_ws(x8, fp8.E4M3, bx, w8, fp8.E4M3, bw, out=y,
+                                  workspace=ws if need > 0 else None)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(device)
+    barrier(world)
+    tot = 0.0
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        b.synchronize()
+        tot += a.elapsed_time(b)
+    ms = max_over_ranks(world, tot / args.steps, device)
+    wbytes = sum(l[0].in_features * l[0].out_features for l in layers)
+    moved = sum(l[0].in_features * l[0].out_features + T * (l[0].in_features * 6 +
+                l[0].out_features * 2) for l in layers)
+    gbs = moved / (ms * 1e-3) / 1e9
+    plans = [fp8.fp8_linear_plan(fp8.FWD, T, l[0].in_features, l[0].out_features,
+                                 with_workspace=l[9] > 0) for l in layers]
+    launches = sum(3 + (1 if p["k_splits"] > 1 else 0) for p in plans)
+    peaks, src = load_peaks()
+    if rank == 0:
+        print(json.dumps({"metric": "decode forward GB/s (weights + activations moved)",
+                          "value": round(gbs * world, 1), "unit": "GB/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": max(3, args.warmup),
+                          "ms_per_step": round(ms, 4), "higher_is_better": True,
+                          "scaling": "weak", "dtype": "fp8", "data": "synthetic",
+                          "config": {"workload": "llama2-70b-proj-decode", "tokens": T,
+                                     "weight_bytes": wbytes,
+                                     "tiles": [[p["tile_m"], p["tile_n"], p["k_splits"]]
+                                               for p in plans],
+                                     "l2": "flushed before each step (outside the timing)"},
+                          "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
+                                       "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                       "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                                       "peak_source": src},
+                          "gpu_launches": launches * args.steps}), flush=True)
+    return 0
+
+
 def run_e2e(args, wl, device, world):
     """Same step through the C ABI from pinned HOST buffers: every step copies
     X, W, dY of each projection in and its Y, dX, dW out (copy streams in both
@@ -531,8 +613,8 @@ def main():
     if not torch.cuda.is_available():
         print(json.dumps({"error": "no CUDA device"}))
         return 1
-    if args.workload == "c4":
-        rc = run_sweep(args, world, rank, local)
+    if args.workload in ("c4", "decode"):
+        rc = (run_sweep if args.workload == "c4" else run_decode)(args, world, rank, local)
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()

@@ -24,6 +24,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -229,18 +231,21 @@ cast_kernel(const uint4* __restrict__ xv, size_t n_items, const void* __restrict
   }
 }
 
-int g_num_sms[64];
+// SM count per device, filled on first use (possibly by several host threads
+// at once, all storing the same value).
+std::atomic<int> g_num_sms[64];
 
 int num_sms() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  if (g_num_sms[dev] == 0) {
-    int n = 0;
+  int n = g_num_sms[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    g_num_sms[dev] = n > 0 ? n : 148;
+    n = n > 0 ? n : 148;
+    g_num_sms[dev].store(n, std::memory_order_relaxed);
   }
-  return g_num_sms[dev];
+  return n;
 }
 
 // Blocks for a streaming kernel over `items` 16-byte vectors: `blocks_per_sm`

@@ -42,6 +42,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -735,16 +737,23 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Host-side caches below (entry point, SM count, co-resident units, scratch
+// address) are filled on first use and may be filled by several host threads
+// at once: they are atomics, and every writer stores the same value (or, for
+// the pair count, the minimum).
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (!f) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess && q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
+            cudaSuccess && q == cudaDriverEntryPointSuccess) {
+      f = reinterpret_cast<EncodeTiledFn>(p);
+      fn.store(f, std::memory_order_release);
+    }
   }
-  return fn;
+  return f;
 }
 
 // 2-D row-major uint8 tensor [outer, inner], box [box_outer, box_inner],
@@ -778,18 +787,19 @@ bool encode_out_2d(CUtensorMap* m, const void* ptr, bool fp32, uint64_t cols, ui
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int g_sm_count[64];
+std::atomic<int> g_sm_count[64];
 
 int sm_count() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  if (g_sm_count[dev] == 0) {
-    int n = 0;
+  int n = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    g_sm_count[dev] = n > 0 ? n : 148;
+    n = n > 0 ? n : 148;
+    g_sm_count[dev].store(n, std::memory_order_relaxed);
   }
-  return g_sm_count[dev];
+  return n;
 }
 
 // Tile order.  Tiles are walked in groups of `group_n` N-blocks, N fastest
@@ -814,17 +824,18 @@ int pick_group_n(uint64_t a_bytes, uint64_t b_bytes) {
 
 // Split K for problems whose tiles cannot fill the GPU (few rows: the
 // weight-streaming GEMMs of decode).  Cut K into ranges so that tiles x splits
-// work units still fit in one wave.  Measured on the Llama-2-70B projections
-// (T = 1 .. 128): splitting pays only for long K ranges and few rows (down,
-// K = 28672, T <= 64: 2.3-3.2 -> 3.6-4.3 TB/s of weights), while short ranges
-// (QKV, K = 8192) and T = 128 lost to the fp32 partial traffic; hence at most
-// 64 rows and at least 48 k-blocks per range.  Returns 1 for no split.
+// work units still fit in one wave, each range at least 16 k-blocks.
+// Measured on the Llama-2-70B projections (T = 1 .. 128, weights streamed,
+// splitk_reduce_kernel summing the partials): QKV (K = 8192) 3.1-3.4 ->
+// 3.7-3.9 TB/s of weights at T <= 64, down (K = 28672) 2.3-3.3 -> 4.1-5.0 TB/s
+// up to T = 128; ranges of >= 24 or >= 48 k-blocks split less and gained less.
+// Returns 1 for no split.
 int plan_splits(int64_t M, int num_tiles, int num_k_blocks, int* kb_per_split) {
   const int sms = sm_count();
   int splits = 1;
-  if (M <= 64 && 2 * num_tiles <= sms) {
+  if (M <= 128 && 2 * num_tiles <= sms) {
     splits = sms / num_tiles;
-    splits = splits < num_k_blocks / 48 ? splits : num_k_blocks / 48;
+    splits = splits < num_k_blocks / 16 ? splits : num_k_blocks / 16;
     splits = splits < 16 ? splits : 16;
     if (splits < 1) splits = 1;
   }
@@ -852,12 +863,19 @@ int plan_pair_splits(int num_tiles, int num_k_blocks, int num_pairs, int* kb_per
 
 // Pairs the pair kernels may run at once on this device: the occupancy query
 // made at their first launch, or one pair per two SMs before that.
-int g_pair_units[64];
+std::atomic<int> g_pair_units[64];
 int pair_units() {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  return g_pair_units[dev] > 0 ? g_pair_units[dev] : sm_count() / 2;
+  const int n = g_pair_units[dev].load(std::memory_order_relaxed);
+  return n > 0 ? n : sm_count() / 2;
+}
+void record_pair_units(int dev, int clusters) {
+  int cur = g_pair_units[dev].load(std::memory_order_relaxed);
+  while ((cur == 0 || clusters < cur) &&
+         !g_pair_units[dev].compare_exchange_weak(cur, clusters, std::memory_order_relaxed)) {
+  }
 }
 
 template <int kTile, bool kAMN, bool kBMN, bool kOutF32, bool kAmax>
@@ -918,7 +936,7 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
   p.amax_out = reinterpret_cast<uint32_t*>(g.d_amax);
   p.wait_limit_ns = kWaitLimitNs;
 
-  static int max_units[64];      // co-resident CTAs (1-CTA) or clusters (pair), per device
+  static std::atomic<int> max_units[64];   // co-resident CTAs (1-CTA) or clusters (pair), per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
@@ -937,7 +955,8 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  if (max_units[dev] == 0) {
+  int units_max = max_units[dev].load(std::memory_order_relaxed);
+  if (units_max == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmem)) != cudaSuccess)
       return FP8_ERR_CUDA;
@@ -950,11 +969,12 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
         clusters = sm_count() / 2;
       }
       units = clusters;
-      if (g_pair_units[dev] == 0 || clusters < g_pair_units[dev]) g_pair_units[dev] = clusters;
+      record_pair_units(dev, clusters);
     }
-    max_units[dev] = units;
+    units_max = units;
+    max_units[dev].store(units, std::memory_order_relaxed);
   }
-  const int units = p.num_work < max_units[dev] ? p.num_work : max_units[dev];
+  const int units = p.num_work < units_max ? p.num_work : units_max;
   cfg.gridDim = dim3(static_cast<unsigned>(units * kCta), 1, 1);
   if (cudaLaunchKernelEx(&cfg, kern, ta, tb, td, p) != cudaSuccess) return FP8_ERR_CUDA;
   if (p.splits > 1) {
@@ -1098,23 +1118,23 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;     // 16 MiB
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 int launch_gemm_noalloc(GemmArgs g, cudaStream_t s) {
-  static void* scratch_addr[64];
+  static std::atomic<void*> scratch_addr[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
-  if (scratch_addr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+  void* scratch = scratch_addr[dev].load(std::memory_order_relaxed);
+  if (scratch == nullptr) {
+    if (cudaGetSymbolAddress(&scratch, g_noalloc_scratch) != cudaSuccess || scratch == nullptr)
       return FP8_ERR_CUDA;
-    scratch_addr[dev] = ptr;
+    scratch_addr[dev].store(scratch, std::memory_order_relaxed);
   }
   size_t need = gemm_workspace_bytes(g);
   if (need > kNoAllocScratchBytes) {
-    if (g.M <= 128) return FP8_ERR_UNSUPPORTED;
-    need = 0;     // CTA-pair tiles: split only when the partials fit, else run unsplit
+    if (g.M <= 64) return FP8_ERR_UNSUPPORTED;
+    need = 0;     // more rows: split only when the partials fit, else run unsplit
   }
   if (need > 0) {
     // every fp32 partial is written by the GEMM before the reduction reads it
-    g.workspace = scratch_addr[dev];
+    g.workspace = scratch;
     g.workspace_bytes = kNoAllocScratchBytes;
   }
   return launch_gemm(g, s);

@@ -152,7 +152,7 @@ fp8_status_t fp8_linear_bwd_dgrad_amax(const uint8_t *dy8, fp8_format_t fdy,
                                        void *stream);
 
 /*
- * fp8_linear_fwd with a split-K workspace.  For few tokens (T <= 64, e.g.
+ * fp8_linear_fwd with a split-K workspace.  For few tokens (T <= 128, e.g.
  * decode-sized inference calls) the GEMM streams the weights and one tile per
  * 128 x 256 block of Y leaves SMs idle; for more tokens, outputs with too few
  * 256 x 256 tiles to fill half the GPU.  With a caller-provided workspace a
@@ -230,11 +230,10 @@ fp8_status_t fp8_linear_plan(fp8_pass_t pass, int64_t T, int64_t in, int64_t out
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
  *   - Nothing is allocated, by this call or below it.
- *   - A problem with T <= 128 whose split-K scratch would exceed 16 MiB
- *     (only possible for T <= 64 with very wide outputs) returns
- *     FP8_ERR_UNSUPPORTED; for T > 128 a split whose partials would not fit
- *     is not made and the forward runs unsplit; problems that do not split
- *     use no scratch at all.
+ *   - A problem with T <= 64 whose split-K scratch would exceed 16 MiB (very
+ *     wide outputs) returns FP8_ERR_UNSUPPORTED; for T > 64 a split whose
+ *     partials would not fit is not made and the forward runs unsplit;
+ *     problems that do not split use no scratch at all.
  *   - All calls share the one array and it keeps the last call's contents:
  *     calls that overlap on the GPU (different streams, no ordering between
  *     them) race on it and must be serialised by the caller.
