@@ -61,6 +61,10 @@ def parse():
                          "the forward of the Llama-2-70B projections for few tokens, weights "
                          "cast once (inference)")
     ap.add_argument("--decode-tokens", type=int, default=16, help="decode: tokens per forward")
+    ap.add_argument("--linears", default=None,
+                    help="c1-c3: comma-separated indices of the projections to run (a subset "
+                         "of the step, e.g. for a profiler capture of one GEMM's real shape "
+                         "with a few GB on the device); default: all of them")
     ap.add_argument("--sweep-log2n", type=int, default=28, help="c4: log2 of the element count")
     ap.add_argument("--sweep-dtype", default="bf16", choices=["bf16", "fp32"])
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -196,13 +200,16 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ the step
 class Workload:
-    def __init__(self, cid, device, seed_step=0, overlap=True, bias_every=1):
+    def __init__(self, cid, device, seed_step=0, overlap=True, bias_every=1, subset=None):
         import fp8_tensor_scaled_b200 as fp8
         from fp8_tensor_scaled_b200.layer import Fp8AmaxStep
         self.cfg = workloads.CONFIGS[cid]
+        self.subset = subset
         self.device = device
         self.inputs, self.layers = [], []
         for li, lin in enumerate(self.cfg.linears):
+            if subset is not None and li not in subset:
+                continue
             x, w, dy = workloads.linear_inputs(cid, li, step=seed_step, device=device)
             self.inputs.append((x, w, dy))
             m = self.cfg.margins[0]
@@ -241,7 +248,9 @@ class Workload:
 def run_fp8(args, world, rank, local):
     device = torch.device("cuda", local)
     cid = int(args.workload[1:])
-    wl = Workload(cid, device, overlap=not args.no_overlap, bias_every=args.bias_every)
+    subset = None if args.linears is None else [int(v) for v in args.linears.split(",")]
+    wl = Workload(cid, device, overlap=not args.no_overlap, bias_every=args.bias_every,
+                  subset=subset)
     stream = torch.cuda.current_stream(device)
     for _ in range(max(3, args.warmup)):
         wl.step()
@@ -592,9 +601,12 @@ def run_reference(args, world, rank):
     return 0
 
 
-def config_dict(cfg, n):
-    return {"workload": cfg.name, "tokens": cfg.tokens,
-            "linears": ["%s %d->%d" % (l.name, l.in_features, l.out_features) for l in cfg.linears],
+def config_dict(cfg, n, subset=None):
+    lins = [l for i, l in enumerate(cfg.linears) if subset is None or i in subset]
+    return {"workload": cfg.name + ("" if subset is None else "-projections-" +
+                                    "-".join(str(i) for i in subset)),
+            "tokens": cfg.tokens,
+            "linears": ["%s %d->%d" % (l.name, l.in_features, l.out_features) for l in lins],
             "passes": list(cfg.passes), "formats": "E4M3 X,W / E5M2 dY", "margin": cfg.margins[0],
             "out_dtype": str(cfg.out_dtype).replace("torch.", ""),
             "l2": "inputs larger than L2 (a step reads and writes several GB)",
@@ -640,7 +652,7 @@ def main():
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8",
-        "data": "synthetic", "config": config_dict(wl.cfg, world),
+        "data": "synthetic", "config": config_dict(wl.cfg, world, wl.subset),
         "gemm_tflops": round(gemm_tflops, 2), "quant_gbs": round(quant_gbs, 1),
         "overlap": not args.no_overlap, "bias_update_every": args.bias_every,
         "launch": "cuda-graph" if args.graph else "eager",
@@ -674,7 +686,7 @@ def main():
                                       "frac": round(e["copy_ms"]["both"] / e["ms_per_step"], 4),
                                       "note": "the step's copies alone, both directions at "
                                               "once, no compute; frac = that time / e2e time"}}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.linears is None:
         cb = oracle_sample(int(args.workload[1:]), args.cpu_seconds)
         line["cpu_baseline"] = {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")}
     if rank == 0:
