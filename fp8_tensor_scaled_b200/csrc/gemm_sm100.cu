@@ -235,16 +235,19 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
   }
 }
 
-// Scale and round one row's 64 accumulator columns (fp32 bits: r0 = columns
-// 0..31, r1 = 32..63) and write them to the warp's staging buffer at `stage`
-// (row `lane`, 128-byte rows, 128-byte swizzle: 16-byte piece j of a row
-// goes to piece j ^ (lane % 8)).  BF16: one 64-column box of 128-byte rows.
-// FP32: two 32-column boxes, the second 4 KB after the first.  With kAmax
-// also fold max |stored| into dmax.
-template <bool kOutF32, bool kAmax>
-__device__ __forceinline__ void stage_out_chunks(uint32_t stage, int lane, const uint32_t (&r0)[32],
-                                                 const uint32_t (&r1)[32], const Pow2Scale& sc,
-                                                 uint32_t& dmax) {
+// 2^e applied as one multiply when e is a normal exponent (the usual case:
+// the whole tile is checked once), else as the split multiplies.
+template <bool kSplit>
+__device__ __forceinline__ float scale_pow2(float x, const Pow2Scale& s) {
+  if (!kSplit) return x * s.f0;
+  return (x * s.f0 * s.f1) * s.f2;
+}
+
+template <bool kOutF32, bool kAmax, bool kSplit>
+__device__ __forceinline__ void stage_out_chunks_t(uint32_t stage, int lane,
+                                                   const uint32_t (&r0)[32],
+                                                   const uint32_t (&r1)[32], const Pow2Scale& sc,
+                                                   uint32_t& dmax) {
   const uint32_t row_base = stage + static_cast<uint32_t>(lane) * 128u;
   const uint32_t sw = static_cast<uint32_t>(lane & 7);
   if (kOutF32) {
@@ -256,7 +259,7 @@ __device__ __forceinline__ void stage_out_chunks(uint32_t stage, int lane, const
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t bits = b == 0 ? r0[4 * j + e] : r1[4 * j + e];
-          w[e] = __float_as_uint(apply_pow2(__uint_as_float(bits), sc));
+          w[e] = __float_as_uint(scale_pow2<kSplit>(__uint_as_float(bits), sc));
           if (kAmax) dmax = max(dmax, w[e] & 0x7FFFFFFFu);
         }
         const uint32_t addr = row_base + static_cast<uint32_t>(b) * 4096u +
@@ -274,7 +277,8 @@ __device__ __forceinline__ void stage_out_chunks(uint32_t stage, int lane, const
         const int col = 8 * j + 2 * e;          // 0..63
         const uint32_t lo = col < 32 ? r0[col] : r1[col - 32];
         const uint32_t hi = col < 32 ? r0[col + 1] : r1[col - 31];
-        w[e] = pack_bf16x2(apply_pow2(__uint_as_float(lo), sc), apply_pow2(__uint_as_float(hi), sc));
+        w[e] = pack_bf16x2(scale_pow2<kSplit>(__uint_as_float(lo), sc),
+                           scale_pow2<kSplit>(__uint_as_float(hi), sc));
         if (kAmax) dmax = __vmaxu2(dmax, w[e] & 0x7FFF7FFFu);
       }
       const uint32_t addr = row_base + ((static_cast<uint32_t>(j) ^ sw) << 4);
@@ -282,6 +286,20 @@ __device__ __forceinline__ void stage_out_chunks(uint32_t stage, int lane, const
                    ::"r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
     }
   }
+}
+
+// Scale and round one row's 64 accumulator columns (fp32 bits: r0 = columns
+// 0..31, r1 = 32..63) and write them to the warp's staging buffer at `stage`
+// (row `lane`, 128-byte rows, 128-byte swizzle: 16-byte piece j of a row
+// goes to piece j ^ (lane % 8)).  BF16: one 64-column box of 128-byte rows.
+// FP32: two 32-column boxes, the second 4 KB after the first.  With kAmax
+// also fold max |stored| into dmax.
+template <bool kOutF32, bool kAmax>
+__device__ __forceinline__ void stage_out_chunks(uint32_t stage, int lane, const uint32_t (&r0)[32],
+                                                 const uint32_t (&r1)[32], const Pow2Scale& sc,
+                                                 uint32_t& dmax) {
+  if (sc.split) stage_out_chunks_t<kOutF32, kAmax, true>(stage, lane, r0, r1, sc, dmax);
+  else          stage_out_chunks_t<kOutF32, kAmax, false>(stage, lane, r0, r1, sc, dmax);
 }
 
 // kAmax: the epilogue also takes the max of |D| over the values it stores
