@@ -518,3 +518,19 @@ def test_concurrent_host_threads():
     for a, b in zip(ref, out):
         for x, y in zip(a, b):
             assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+def test_unscale_exponent_beyond_normal_range(out_dtype):
+    """Tiny tensors give biases near 66 (E4M3) and 73 (E5M2), so the GEMM's
+    unscale 2^-(bA+bB) has an exponent below -126, outside what one fp32
+    power of two holds: the epilogue applies it as split multiplies.  The
+    products stay normal numbers, so the results are compared in full."""
+    T, In, Out = 200, 272, 400
+    x, w, dy = _inputs(T, In, Out, seed=77, x_scale=2.0 ** -60, w_scale=2.0 ** -60,
+                       dy_scale=2.0 ** -60)
+    Q = _passes(x, w, dy)
+    bx, bw, bdy = Q["x"][3], Q["w"][3], Q["dy"][3]
+    assert bx + bw > 127 and bdy + bw > 127 and bdy + bx > 127, (bx, bw, bdy)
+    for p in (oracle.FWD, oracle.DGRAD, oracle.WGRAD):
+        _compare_full(p, Q, T, In, Out, out_dtype, "split unscale pass %d" % p)
