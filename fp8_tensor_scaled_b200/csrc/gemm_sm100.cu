@@ -18,18 +18,20 @@
 //   problems of many tiles use 256 x 512 tiles (two such MMAs per K step that
 //   share the A stage: a quarter less L2 traffic per FLOP).
 //   warp 0      TMA producer: 128 x 128-byte FP8 boxes with 128-byte swizzle
-//               (no multicast: each CTA loads its own halves) into a 6-stage
-//               shared-memory ring of 32 KB stages (4 x 48 KB for one CTA);
-//               the pair's copies complete on the leader's mbarrier, armed
-//               with the bytes of both CTAs.
+//               (no multicast: each CTA loads its own halves) into a ring of
+//               192 KB per CTA (6 x 32 KB for 256 x 256 tiles, 4 x 48 KB for
+//               256 x 512 and 128 x 256 tiles); the pair's copies complete on
+//               the leader's mbarrier, armed with the bytes of both CTAs.
 //   warp 1      TMEM allocator (512 columns = two 128 x 256 fp32 accumulators
-//               per CTA, or one 128 x 512 for 256 x 512 tiles); in the leader, one thread issues the MMAs (four per
-//               stage) and tcgen05.commit, multicast to both CTAs' barriers,
-//               frees each stage and publishes each finished accumulator.
+//               per CTA, or one 128 x 512 for 256 x 512 tiles); in the
+//               leader, one thread issues the MMAs and tcgen05.commit,
+//               multicast to both CTAs' barriers, which frees each stage and
+//               publishes each finished accumulator.
 //   warps 2-5   epilogue: tcgen05.ld 32x32b of the CTA's accumulator rows,
 //               multiply by the power of two 2^-(bias_a+bias_b), one rounding
-//               to BF16/FP32, 16-byte stores; two accumulators let it overlap
-//               the next tile's mainloop.
+//               to BF16/FP32 into a swizzled shared-memory box, one TMA store
+//               per box.  Two accumulators (or two halves of one) let it
+//               overlap the next tile's mainloop.
 // Tiles are visited in groups of 16 N-blocks, N fastest inside a group, so
 // that the clusters running at one time share A and B panels in L2.
 //
