@@ -174,13 +174,21 @@ class Fp8AmaxStep:
         return sum(l.flops() for l in self.linears)
 
     def _quantize(self, i, inputs, after=None, timing=None):
+        """Quantize linear i's X, W (and dY) in that order on the quantization
+        stream, recording an event after each tensor (t_q[i][t]) so that a
+        pass can start as soon as its own two operands are ready."""
         stream = self.side if self.overlap else torch.cuda.current_stream(self.device)
+        lin = self.linears[i]
+        L = Fp8AmaxLinear
         with torch.cuda.stream(stream):
             if after is not None:
                 stream.wait_event(after)
             if timing is not None:
                 timing["q"][i][0].record(stream)
-            self.linears[i].quantize(*inputs[i])
+            refresh = lin.begin_step()
+            for t in ((L.X, L.W, L.DY) if lin.backward else (L.X, L.W)):
+                lin.quantize_one(t, inputs[i][t], refresh)
+                self.t_q[i][t].record(stream)
             if timing is not None:
                 timing["q"][i][1].record(stream)
             self.q_done[i].record(stream)
@@ -194,14 +202,22 @@ class Fp8AmaxStep:
         n = len(self.linears)
         # linear 0 is quantized first; every later one while the previous GEMMs run
         self._quantize(0, inputs, after=in_events[0] if in_events else start, timing=timing)
+        L = Fp8AmaxLinear
         for i in range(n):
             if i + 1 < n:
                 self._quantize(i + 1, inputs, after=in_events[i + 1] if in_events else None,
                                timing=timing)
-            main.wait_event(self.q_done[i])
-            if timing is not None:
-                timing["g"][i][0].record(main)
-            self.linears[i].gemms(self.p_done[i])
+            lin = self.linears[i]
+            passes = (L.FWD, L.DGRAD, L.WGRAD) if lin.backward else (L.FWD,)
+            for j, k in enumerate(passes):
+                # each pass waits only for its own operands: the forward of
+                # the first linear runs while its dY is still being quantized
+                for t in L.PASS_INPUTS[k]:
+                    main.wait_event(self.t_q[i][t])
+                if j == 0 and timing is not None:
+                    timing["g"][i][0].record(main)
+                lin.gemm(k)
+                self.p_done[i][k].record(main)
             if timing is not None:
                 timing["g"][i][1].record(main)
             self.g_done[i].record(main)
