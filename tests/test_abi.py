@@ -77,3 +77,36 @@ def test_empty_token_count_is_valid_shape(L):
     # T == 0 passes argument checks with null token-sized tensors (then needs a device)
     r = L.fp8_linear_fwd(P(0), 0, A16, A16, 0, A16, 0, 32, 32, P(0), 0, P(0))
     assert r in (OK, NO_DEVICE)
+
+
+def test_workspace_and_plan_entry_points(L):
+    """Argument checks of the workspace, no-allocation and plan entry points
+    run before any device work."""
+    i64, sz = ctypes.c_int64, ctypes.c_size_t
+    ws = lambda wptr, wbytes, y=A16: (A16, 0, A16, A16, 0, A16, i64(128), i64(32), i64(32), y, 0,
+                                      wptr, sz(wbytes), P(0))
+    # a workspace must be 256-byte aligned, and non-null when bytes are given
+    assert L.fp8_linear_fwd_ws(*ws(P(0x10010), 1024)) == MISALIGNED
+    assert L.fp8_linear_fwd_ws(*ws(P(0), 1024)) == INVALID
+    assert L.fp8_linear_fwd_ws(*ws(P(0x10000), 1024, y=P(0x10008))) == MISALIGNED
+    assert L.fp8_linear_bwd_wgrad_ws(*ws(P(0x10010), 1024)) == MISALIGNED
+    assert L.fp8_linear_bwd_wgrad_ws(*ws(P(0), 1024)) == INVALID
+    f = L.fp8_linear_fwd_noalloc
+    f.argtypes = [P, ctypes.c_int, P, P, ctypes.c_int, P, i64, i64, i64, P, ctypes.c_int, P]
+    f.restype = ctypes.c_int
+    assert f(A16, 0, A16, A16, 0, A16, 128, 17, 32, A16, 0, P(0)) == UNSUPPORTED
+    assert f(A16, 0, A16, A16, 0, A16, 128, 32, 32, P(0x10008), 0, P(0)) == MISALIGNED
+    # the size queries report 0 without a device (nothing to plan on)
+    if not torch.cuda.is_available():
+        assert L.fp8_linear_fwd_workspace_size(16, 12288, 512) == 0
+        assert L.fp8_linear_bwd_wgrad_workspace_size(8192, 768, 768) == 0
+    # the plan query: null plan, unknown pass, negative sizes -> INVALID
+    g = L.fp8_linear_plan
+    g.argtypes = [ctypes.c_int, i64, i64, i64, ctypes.c_int, P]
+    g.restype = ctypes.c_int
+    plan = (ctypes.c_int32 * 4)()
+    assert g(0, 16, 16, 16, 0, P(0)) == INVALID
+    assert g(3, 16, 16, 16, 0, ctypes.cast(plan, P)) == INVALID
+    assert g(0, -1, 16, 16, 0, ctypes.cast(plan, P)) == INVALID
+    if not torch.cuda.is_available():
+        assert g(0, 16, 16, 16, 0, ctypes.cast(plan, P)) == NO_DEVICE
