@@ -77,8 +77,6 @@ template <bool kBF16>
 __global__ void __launch_bounds__(kThreads)
 amax_kernel(const uint4* __restrict__ xv, size_t n_vec, const void* __restrict__ tail,
             uint32_t n_tail, uint32_t* __restrict__ amax_bits) {
-  pdl_wait();
-  pdl_trigger();
   uint32_t m = 0;  // for bf16: two packed 16-bit |x| maxima
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -140,8 +138,6 @@ amax_kernel(const uint4* __restrict__ xv, size_t n_vec, const void* __restrict__
 // --------------------------------------------------------------------------
 __global__ void compute_bias_kernel(const uint32_t* __restrict__ amax_bits, int fmt,
                                     int32_t margin, int32_t* __restrict__ bias) {
-  pdl_wait();
-  pdl_trigger();
   *bias = bias_from_amax_bits(*amax_bits, fmt, margin);
 }
 
@@ -190,8 +186,6 @@ cast_kernel(const uint4* __restrict__ xv, size_t n_items, const void* __restrict
             uint32_t n_tail, const int32_t* __restrict__ bias_in,
             const uint32_t* __restrict__ amax_bits, int32_t margin, int32_t* __restrict__ bias_out,
             uint8_t* __restrict__ out) {
-  pdl_wait();
-  pdl_trigger();
   int32_t bias;
   if (kFromAmax) {
     bias = bias_from_amax_bits(*amax_bits, kFmt, margin);
@@ -278,21 +272,18 @@ cudaError_t launch_amax(const void* x, int dt, size_t n, float* amax, cudaStream
   const void* tail = static_cast<const uint8_t*>(x) + n_vec * per_vec * esz;
   const unsigned grid = grid_for(n_vec, kAmaxUnroll, kAmaxBlocksPerSm);
   if (dt == FP8_DTYPE_BF16)
-    e = launch_pdl(amax_kernel<true>, dim3(grid), dim3(kThreads), 0, s,
-                   static_cast<const uint4*>(x), n_vec, tail, n_tail,
-                   reinterpret_cast<uint32_t*>(amax));
+    amax_kernel<true><<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(x), n_vec, tail, n_tail,
+                                                reinterpret_cast<uint32_t*>(amax));
   else
-    e = launch_pdl(amax_kernel<false>, dim3(grid), dim3(kThreads), 0, s,
-                   static_cast<const uint4*>(x), n_vec, tail, n_tail,
-                   reinterpret_cast<uint32_t*>(amax));
-  return e != cudaSuccess ? e : cudaGetLastError();
+    amax_kernel<false><<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(x), n_vec, tail, n_tail,
+                                                 reinterpret_cast<uint32_t*>(amax));
+  return cudaGetLastError();
 }
 
 cudaError_t launch_compute_bias(const float* amax, int fmt, int32_t margin, int32_t* bias,
                                 cudaStream_t s) {
-  const cudaError_t e = launch_pdl(compute_bias_kernel, dim3(1), dim3(1), 0, s,
-                                   reinterpret_cast<const uint32_t*>(amax), fmt, margin, bias);
-  return e != cudaSuccess ? e : cudaGetLastError();
+  compute_bias_kernel<<<1, 1, 0, s>>>(reinterpret_cast<const uint32_t*>(amax), fmt, margin, bias);
+  return cudaGetLastError();
 }
 
 namespace {
@@ -307,14 +298,13 @@ cudaError_t launch_cast_t(const void* x, size_t n, int fmt, const int32_t* bias_
   const unsigned grid = grid_for(n_items, kCastUnroll, kCastBlocksPerSm);
   const uint4* xv = static_cast<const uint4*>(x);
   const uint32_t* ab = reinterpret_cast<const uint32_t*>(amax);
-  cudaError_t e;
   if (fmt == FP8_E4M3)
-    e = launch_pdl(cast_kernel<kBF16, FP8_E4M3, kFromAmax>, dim3(grid), dim3(kThreads), 0, s,
-                   xv, n_items, tail, n_tail, bias_in, ab, margin, bias_out, out);
+    cast_kernel<kBF16, FP8_E4M3, kFromAmax><<<grid, kThreads, 0, s>>>(
+        xv, n_items, tail, n_tail, bias_in, ab, margin, bias_out, out);
   else
-    e = launch_pdl(cast_kernel<kBF16, FP8_E5M2, kFromAmax>, dim3(grid), dim3(kThreads), 0, s,
-                   xv, n_items, tail, n_tail, bias_in, ab, margin, bias_out, out);
-  return e != cudaSuccess ? e : cudaGetLastError();
+    cast_kernel<kBF16, FP8_E5M2, kFromAmax><<<grid, kThreads, 0, s>>>(
+        xv, n_items, tail, n_tail, bias_in, ab, margin, bias_out, out);
+  return cudaGetLastError();
 }
 }  // namespace
 

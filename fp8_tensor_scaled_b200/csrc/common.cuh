@@ -100,18 +100,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Programmatic dependent launch.  A kernel launched with programmatic stream
-// serialization may be scheduled before the previous kernel of its stream has
-// finished: pdl_wait() blocks until that kernel has completed and its memory
-// operations are visible (it returns at once when there is no such
-// predecessor), so every kernel calls it before it reads or writes global
-// memory.  pdl_trigger() allows the next such kernel of the stream to be
-// scheduled once every block of this one has called it (or exited).
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_trigger() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory, MMA, commit, loads, fences
 // ---------------------------------------------------------------------------

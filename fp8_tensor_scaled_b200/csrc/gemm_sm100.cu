@@ -381,9 +381,6 @@ fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
   else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // everything above (barriers, tensor memory, descriptor prefetch) may
-  // overlap the previous kernel of the stream; global memory only after it
-  pdl_wait();
 
   if (warp == 0 && lane == 0) {
     // ----------------------------- TMA producer -----------------------------
@@ -709,8 +706,6 @@ template <bool kOutF32, bool kAmax>
 __global__ void __launch_bounds__(kReduceThreads)
 splitk_reduce_kernel(const float4* __restrict__ ws, int splits, int64_t n4,
                      const int32_t* bias_a, const int32_t* bias_b, void* d, uint32_t* amax_out) {
-  pdl_wait();
-  pdl_trigger();
   const Pow2Scale sc = make_pow2_scale(-(*bias_a + *bias_b));
   uint32_t dmax = 0;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -968,7 +963,7 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
   auto kern = fp8_gemm_kernel<kTile, kAMN, kBMN, kOutF32, kAmax>;
 
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
@@ -1001,20 +996,15 @@ int launch_t(const GemmArgs& g, cudaStream_t s) {
   }
   const int units = p.num_work < units_max ? p.num_work : units_max;
   cfg.gridDim = dim3(static_cast<unsigned>(units * kCta), 1, 1);
-  attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs += 1;
   if (cudaLaunchKernelEx(&cfg, kern, ta, tb, td, p) != cudaSuccess) return FP8_ERR_CUDA;
   if (p.splits > 1) {
     const int64_t n4 = static_cast<int64_t>(g.M) * g.N / 4;
     int64_t blocks = (n4 + kReduceThreads - 1) / kReduceThreads;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
     if (blocks > cap) blocks = cap;
-    if (launch_pdl(splitk_reduce_kernel<kOutF32, kAmax>, dim3(static_cast<unsigned>(blocks)),
-                   dim3(kReduceThreads), 0, s, reinterpret_cast<const float4*>(p.ws), p.splits,
-                   n4, g.bias_a, g.bias_b, g.d, p.amax_out) != cudaSuccess)
-      return FP8_ERR_CUDA;
+    splitk_reduce_kernel<kOutF32, kAmax><<<static_cast<unsigned>(blocks), kReduceThreads, 0, s>>>(
+        reinterpret_cast<const float4*>(p.ws), p.splits, n4, g.bias_a, g.bias_b, g.d,
+        p.amax_out);
   }
   return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }

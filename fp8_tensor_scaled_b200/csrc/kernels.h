@@ -7,26 +7,6 @@
 
 namespace fp8amax {
 
-// Launch `kern` on `s` with programmatic stream serialization: the kernel may
-// be scheduled while the previous kernel of the stream finishes, and waits for
-// it with pdl_wait() (every kernel of this library does so before touching
-// global memory).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t s, Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-}
-
 cudaError_t launch_amax(const void* x, int dt, size_t n, float* amax, cudaStream_t s);
 cudaError_t launch_compute_bias(const float* amax, int fmt, int32_t margin, int32_t* bias,
                                 cudaStream_t s);
